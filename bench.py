@@ -1,0 +1,485 @@
+"""Benchmark of the FibQuant KV codec hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fibquant|reference]
+                    [--workload gpt2|tinyllama|large|toy]
+
+One step = one pass of the whole hot path over the workload's synthetic GPT-2-small-shaped
+KV cache (12 layers x 12 heads x 1024 tokens, K and V, d = 64, fp16): for each of its two
+rates (k=3 N=64 with the exact grid search, k=4 N=8 with brute force) encode K and V
+(separate rotations) and decode K and V to fp16.  The metric is fp16-equivalent GB/s:
+(encode input + decode output) bytes as an fp16 cache, divided by the step time.  The fused
+decode-attention step (B16, Hq32/Hkv4, T32768, d64) is timed in the same run and reported
+under "attn".  Inputs rotate over enough copies that every kernel reads data that has left
+the 126 MB L2 (the whole-step footprint between reuses is >= 2x L2).
+
+With --gpus N > 1 (launched by torch.distributed.run), every rank processes its own cache of
+the same shape (weak scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import glob
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from random_access_kv_fq_b200 import workloads as wl  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+WORKLOADS = {"gpt2": wl.GPT2, "tinyllama": wl.TINYLLAMA, "large": wl.LARGE, "toy": wl.TOY}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "random_access_kv_fq_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_label: str):
+    """Per-launch DRAM bytes recorded from an ncu capture of this exact source, else None."""
+    for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        for line in open(f):
+            m = re.match(r"traffic\s+(\S+)\s+bytes_per_launch=(\d+)\s+source_sha=(\w+)", line)
+            if m and m.group(1) == kernel_label and m.group(3) == source_sha():
+                return int(m.group(2))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workload setup
+
+@dataclasses.dataclass
+class RateState:
+    rate: wl.Rate
+    rot: dict        # tensor -> device rotation
+    cb: object
+    index: object
+    P: int
+    codes: list      # per copy: [n, P] uint8
+    norms: list      # per copy: [n] int16
+
+
+def build_codec_state(torch, fq, w, rank, copies, device):
+    shape = dataclasses.replace(w.cache, seed=w.cache.seed + 7919 * rank)
+    n, d = shape.n, shape.d
+    half = n // 2
+    host = wl.cache(shape)
+    tdtype = torch.float16 if shape.dtype == "f16" else torch.float32
+    xs = [torch.from_numpy(host).to(device) for _ in range(copies)]
+    from random_access_kv_fq_b200 import tables
+    states = []
+    for rate in w.rates:
+        dp = fq.fq_padded_dim(d, rate.k)
+        rot = {"K": torch.from_numpy(tables.rotation(dp, wl.ROT_SEED_K)).to(device),
+               "V": torch.from_numpy(tables.rotation(dp, wl.ROT_SEED_V)).to(device)}
+        cb_np = tables.codebook(dp, rate.k, rate.N)
+        cb = torch.from_numpy(cb_np).to(device)
+        index = None
+        if rate.search != "brute":
+            kind = fq.FQ_INDEX_EXACT if rate.search == "exact" else fq.FQ_INDEX_TOPC
+            index = torch.from_numpy(fq.fq_build_search_index(cb_np, d, rate.k, rate.N, kind,
+                                                              rate.grid_L, rate.grid_c)).to(device)
+        P = fq.fq_payload_bytes(d, rate.k, rate.N)
+        codes = [torch.empty((n, P), dtype=torch.uint8, device=device) for _ in range(copies)]
+        norms = [torch.empty((n,), dtype=torch.int16, device=device) for _ in range(copies)]
+        st = RateState(rate, rot, cb, index, P, codes, norms)
+        for c in range(copies):  # valid records everywhere before timing
+            for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
+                fq.fq_encode(xs[c][sl], rot[t], cb, rate.k, rate.N, codes=codes[c][sl],
+                             norms=norms[c][sl], search_index=index)
+        states.append(st)
+    ys = [torch.empty((n, d), dtype=torch.float16, device=device) for _ in range(copies)]
+    torch.cuda.synchronize()
+    return shape, host, xs, ys, states
+
+
+def codec_launches(fq, shape, xs, ys, states, c, prev):
+    """The launches of one step on copy c (decode reads the records of copy `prev`).  Yields
+    (label, kind, algorithmic bytes, fp16-equivalent bytes, launch thunk)."""
+    n, d = shape.n, shape.d
+    half = n // 2
+    for st in states:
+        r = st.rate
+        for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
+            nv = sl.stop - sl.start
+            xb = xs[c].element_size() * d
+            yield (f"encode_{r.label}", "encode", nv * (xb + st.P + 2), nv * 2 * d,
+                   lambda st=st, t=t, sl=sl: fq.fq_encode(
+                       xs[c][sl], st.rot[t], st.cb, st.rate.k, st.rate.N, codes=st.codes[c][sl],
+                       norms=st.norms[c][sl], search_index=st.index))
+            yield (f"decode_{r.label}", "decode", nv * (st.P + 2 + 2 * d), nv * 2 * d,
+                   lambda st=st, t=t, sl=sl: fq.fq_decode(
+                       st.codes[prev][sl], st.norms[prev][sl], st.rot[t], st.cb, d, st.rate.k,
+                       st.rate.N, y=ys[c][sl]))
+
+
+def attn_state(torch, fq, device, copies, rank):
+    w = wl.ATTN
+    from random_access_kv_fq_b200 import tables
+    dpk, dpv = fq.fq_padded_dim(w.d, w.k_rate.k), fq.fq_padded_dim(w.d, w.v_rate.k)
+    rk = torch.from_numpy(tables.rotation(dpk, wl.ROT_SEED_K)).to(device)
+    rv = torch.from_numpy(tables.rotation(dpv, wl.ROT_SEED_V)).to(device)
+    ck = torch.from_numpy(tables.codebook(dpk, w.k_rate.k, w.k_rate.N)).to(device)
+    cv = torch.from_numpy(tables.codebook(dpv, w.v_rate.k, w.v_rate.N)).to(device)
+    q = torch.from_numpy(wl.attn_queries(w)).to(device)
+    kx = torch.from_numpy(wl.attn_kv(w, "K").reshape(-1, w.d)).to(device)
+    vx = torch.from_numpy(wl.attn_kv(w, "V").reshape(-1, w.d)).to(device)
+    kc, kn = fq.fq_encode(kx, rk, ck, w.k_rate.k, w.k_rate.N)
+    vc, vn = fq.fq_encode(vx, rv, cv, w.v_rate.k, w.v_rate.N)
+    del kx, vx
+    shp = (w.batch, w.hkv, w.tokens)
+    kcs = [kc.reshape(*shp, -1).clone() for _ in range(copies)]
+    kns = [kn.reshape(shp).clone() for _ in range(copies)]
+    vcs = [vc.reshape(*shp, -1).clone() for _ in range(copies)]
+    vns = [vn.reshape(shp).clone() for _ in range(copies)]
+    ws = torch.empty((fq.fq_attn_workspace_bytes(w.batch, w.hq, w.hkv, w.tokens, w.d,
+                                                 w.v_rate.k),), dtype=torch.uint8, device=device)
+    out = torch.empty((w.batch, w.hq, w.d), dtype=torch.float32, device=device)
+    step_bytes = w.batch * w.hkv * w.tokens * (kcs[0].shape[-1] + 2 + vcs[0].shape[-1] + 2)
+
+    def launch(c):
+        fq.fq_attn_decode(q, kcs[c], kns[c], w.k_rate.k, w.k_rate.N, rk, ck, vcs[c], vns[c],
+                          w.v_rate.k, w.v_rate.N, rv, cv, scale=1 / math.sqrt(w.d), out=out,
+                          workspace=ws)
+    return launch, step_bytes
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_gpu(args):
+    import torch
+    import random_access_kv_fq_b200 as fq
+    fq.lib()  # fail loudly when the CUDA library is missing
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    shape0 = w.cache
+    step_bytes_est = shape0.n * (shape0.d * 2) * 3 * len(w.rates)
+    copies = max(2, math.ceil(2 * L2_BYTES / max(step_bytes_est, 1)) + 1)
+    copies = min(copies, 8)
+    shape, host, xs, ys, states = build_codec_state(torch, fq, w, rank, copies, device)
+    attn_launch, attn_bytes = attn_state(torch, fq, device, 4, rank) if not args.no_attn else (None, 0)
+    n_launch = sum(1 for _ in codec_launches(fq, shape, xs, ys, states, 0, 0))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    # warm-up
+    for i in range(args.warmup):
+        c = i % copies
+        for lab, kind, ab, eb, fn in codec_launches(fq, shape, xs, ys, states, c, (c - 1) % copies):
+            fn()
+        if attn_launch:
+            attn_launch(i % 4)
+    barrier()
+    # timed region: K steps, per-launch events on the launching stream
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_launch)] for _ in range(args.steps)]
+    meta = None
+    with ClockSampler(local) as clk:
+        barrier()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            c = i % copies
+            launches = list(codec_launches(fq, shape, xs, ys, states, c, (c - 1) % copies))
+            if meta is None:
+                meta = [(lab, kind, ab, eb) for lab, kind, ab, eb, _ in launches]
+            for j, (_, _, _, _, fn) in enumerate(launches):
+                ev[i][j][0].record(stream)
+                fn()
+                ev[i][j][1].record(stream)
+        t_end.record(stream)
+        barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    per = {}
+    for i in range(args.steps):
+        for j, (lab, kind, ab, eb) in enumerate(meta):
+            ms = ev[i][j][0].elapsed_time(ev[i][j][1])
+            s = per.setdefault(lab, {"ms": 0.0, "launches": 0, "alg_bytes": ab, "kind": kind,
+                                     "eq_bytes": 0})
+            s["ms"] += ms
+            s["launches"] += 1
+    step_eq = sum(eb for _, _, _, eb in meta)
+    value = world * step_eq * args.steps / (total_ms * 1e-3) / 1e9
+    hbm, hbm_src = peaks()
+    dom_lab = max(per, key=lambda k: per[k]["ms"])
+    dom = per[dom_lab]
+    avg_ms = dom["ms"] / dom["launches"]
+    achieved = dom["alg_bytes"] / (avg_ms * 1e-3) / 1e9
+    kernels = {lab: {"avg_us": round(1e3 * s["ms"] / s["launches"], 2),
+                     "GBps_alg": round(s["alg_bytes"] / (s["ms"] / s["launches"] * 1e-3) / 1e9, 1),
+                     "share": round(s["ms"] / sum(v["ms"] for v in per.values()), 3)}
+               for lab, s in per.items()}
+    result = {
+        "metric": "KV encode/decode GB/s (fp16-equiv) & % of roofline; fused attn us/step",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16->u8/fp32",
+        "data": "synthetic (seeded; GPT-2-small-shaped KV cache recipe, no weights)",
+        "config": {"workload": w.name, "vectors_per_gpu": shape.n, "d": shape.d,
+                   "rates": [r.label for r in w.rates], "decode_out": "fp16",
+                   "l2": f"inputs rotate over {copies} copies (>= 2x L2 between reuses)",
+                   "step": "encode K,V + decode K,V per rate"},
+        "roofline": {"bound": "hbm", "kernel": dom_lab, "achieved": round(achieved, 1),
+                     "peak": hbm, "peak_source": hbm_src, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": profiled_traffic(dom_lab),
+                     "alg_bytes_per_launch": dom["alg_bytes"]},
+        "kernels": kernels,
+        "gpu_launches": None,
+        "clocks": clk.summary(),
+    }
+    launches_per_step = sum(1 for _ in meta)
+    gpu_launches = launches_per_step * args.steps
+    # fused attention step
+    if attn_launch:
+        reps = max(20, args.steps // 10)
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(reps):
+            attn_launch(i % 4)
+        a1.record(stream)
+        barrier()
+        us = a0.elapsed_time(a1) * 1e3 / reps
+        result["attn"] = {"workload": wl.ATTN.name, "us_per_step": round(us, 2),
+                          "bytes_per_step": attn_bytes,
+                          "roofline": {"bound": "hbm", "achieved": round(attn_bytes / (us * 1e-6) / 1e9, 1),
+                                       "peak": hbm, "unit": "GB/s",
+                                       "frac": round(attn_bytes / (us * 1e-6) / 1e9 / hbm, 4)},
+                          "launches_per_step": 2}
+    result["gpu_launches"] = gpu_launches
+    # end to end through the public API with pinned host buffers
+    if not args.no_e2e:
+        result["e2e"] = e2e(torch, fq, shape, host, states, args, device, world, dist)
+    if rank == 0:
+        result["cpu_baseline"] = cpu_baseline(w, args) if not args.no_cpu else None
+        print(json.dumps(result), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e(torch, fq, shape, host, states, args, device, world, dist):
+    """Same metric through the public API with host buffers: every step copies the pinned
+    host cache in, encodes, copies the records out, copies records in, decodes, copies the
+    fp16 result out."""
+    n, d = shape.n, shape.d
+    half = n // 2
+    xh = torch.from_numpy(host).pin_memory()
+    xd = torch.empty_like(xh, device=device)
+    outs = []
+    for st in states:
+        outs.append((torch.empty((n, st.P), dtype=torch.uint8).pin_memory(),
+                     torch.empty((n,), dtype=torch.int16).pin_memory()))
+    yh = torch.empty((n, d), dtype=torch.float16).pin_memory()
+    yd = torch.empty((n, d), dtype=torch.float16, device=device)
+    h2d = d2h = 0
+
+    def step():
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+        xd.copy_(xh, non_blocking=True)
+        h2d += xh.numel() * xh.element_size()
+        for st, (ch, nh) in zip(states, outs):
+            cd, nd = st.codes[0], st.norms[0]
+            for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
+                fq.fq_encode(xd[sl], st.rot[t], st.cb, st.rate.k, st.rate.N, codes=cd[sl],
+                             norms=nd[sl], search_index=st.index)
+            ch.copy_(cd, non_blocking=True)
+            nh.copy_(nd, non_blocking=True)
+            d2h += ch.numel() + nh.numel() * 2
+            cd2, nd2 = st.codes[1], st.norms[1]
+            cd2.copy_(ch, non_blocking=True)
+            nd2.copy_(nh, non_blocking=True)
+            h2d += ch.numel() + nh.numel() * 2
+            for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
+                fq.fq_decode(cd2[sl], nd2[sl], st.rot[t], st.cb, d, st.rate.k, st.rate.N, y=yd[sl])
+            yh.copy_(yd, non_blocking=True)
+            d2h += yh.numel() * 2
+
+    for _ in range(max(3, args.warmup // 10)):
+        step()
+    torch.cuda.synchronize()
+    reps = max(5, min(50, args.steps // 20))
+    if dist is not None:
+        dist.barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(reps):
+        step()
+    s1.record()
+    torch.cuda.synchronize()
+    ms = s0.elapsed_time(s1)
+    if dist is not None:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    eq = 2 * n * 2 * d * len(states)
+    return {"value": round(world * eq * reps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": reps}
+
+
+def cpu_baseline(w, args, budget_s: float = 12.0):
+    """The CPU oracle, as it stands, timed on this host on a bounded sample of the workload
+    (single BLAS thread)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import fq_oracle as fo
+    from random_access_kv_fq_b200 import tables
+    shape = w.cache
+    rng = np.random.default_rng(0)
+    sample = np.sort(rng.choice(shape.n, size=min(2048, shape.n), replace=False))
+    x = wl.rows_of(shape, sample)
+    done_eq = 0
+    t0 = time.perf_counter()
+    with threadpool_limits(1):
+        while time.perf_counter() - t0 < budget_s:
+            for rate in w.rates:
+                dp = fo.padded_dim(shape.d, rate.k)
+                rot = tables.rotation(dp, wl.ROT_SEED_K)
+                cb = tables.codebook(dp, rate.k, rate.N)
+                enc = fo.encode(x, rot, cb, rate.k)
+                codes = fo.pack(enc.idx, rate.N)
+                fo.decode(codes, enc.norms, rot, cb, shape.d, rate.k, rate.N)
+                done_eq += 2 * x.shape[0] * 2 * shape.d
+    el = time.perf_counter() - t0
+    return {"value": round(done_eq / el / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{x.shape[0]} sampled vectors of {w.name}, encode+pack+decode at every "
+                      f"rate, repeated for {el:.1f} s (fp64 NumPy, 1 thread)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    cb = cpu_baseline(w, args, budget_s=max(3.0, min(20.0, 2.0 * args.steps)))
+    line = {"impl": "reference", "metric": "KV encode/decode GB/s (fp16-equiv) & % of roofline; "
+            "fused attn us/step", "value": cb["value"], "unit": "GB/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "rates": [r.label for r in w.rates]},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="fibquant", choices=["fibquant", "reference"])
+    ap.add_argument("--workload", default="gpt2", choices=list(WORKLOADS))
+    ap.add_argument("--no-attn", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,157 @@
+/*
+ * fq.h - C ABI of the FibQuant KV-cache codec for NVIDIA B200 (sm_100a).
+ *
+ * FibQuant ("FibQuant: Universal Vector Quantization for Random-Access KV-Cache Compression",
+ * technical summary sec. 2.3) encodes a key or value vector x in R^d as
+ *   - its norm nu = |x|_2 (stored as IEEE fp16, round to nearest even),
+ *   - the unit vector rotated by one shared Haar matrix, z = Pi x / nu,
+ *   - split into m = d'/k blocks of k consecutive coordinates, each replaced by the index of
+ *     its nearest codeword in one shared codebook of N codewords (B = log2 N bits each).
+ * The decoder fetches the codewords, concatenates them, applies Pi^T and scales by nu.
+ * Records are fixed-size so that any token decodes alone by address arithmetic (summary
+ * sec. 1, "random access").
+ *
+ * Notation used below:  d = vector length; k = block size; d' = k * ceil(d / k) (x is
+ * zero-padded to d' when k does not divide d); m = d' / k; N = codebook size, a power of two
+ * in [2, 65536]; B = log2 N; P = ceil(m * B / 8) = fq_payload_bytes(d, k, N).
+ *
+ * Record layout (a fixed-rate, fixed-address format, two planes):
+ *   codes plane: n records of P bytes, record t at byte offset t * P.  Index j of a record
+ *                occupies record bits [j*B, (j+1)*B), least significant bit first; record bit
+ *                i is bit (i % 8) of byte (i / 8); unused tail bits are zero.
+ *   norms plane: n IEEE fp16 values (passed as uint16_t bit patterns), norm t at element t.
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers unless the comment says "host".  The caller owns
+ *     every buffer; the library never allocates device memory and keeps no state between calls.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) and is
+ *     asynchronous; results are valid once the stream has reached the enqueued work.
+ *   - Errors are returned as fq_status from host-side validation before anything is enqueued,
+ *     or FQ_ERR_CUDA when a launch fails.  Nothing aborts or throws across the ABI.
+ *   - n = 0 (or T = 0 in attention) is a valid no-op returning FQ_OK.
+ *   - Limits: 1 <= d <= 256, 1 <= k <= 8, k <= d, N a power of two in [2, 65536]; other
+ *     values return FQ_ERR_UNSUPPORTED.  Non-finite inputs are a precondition violation and
+ *     are not detected.
+ *   - Rotation `rot`: d' x d' fp32, row-major, z = rot * pad(x) (rows = output coordinates).
+ *     Codebook `codebook`: N x k fp32, row-major.  Both are plain input data; the library
+ *     reads them on every call (they are small: at most 256 KB and 2 MB).
+ */
+#ifndef FQ_H_
+#define FQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FQ_OK = 0,
+  FQ_ERR_INVALID_ARG = 1, /* null pointer for a non-empty call, negative size, bad enum */
+  FQ_ERR_UNSUPPORTED = 2, /* a size outside the limits above */
+  FQ_ERR_ALIGNMENT = 3,   /* a pointer that breaks a stated alignment rule */
+  FQ_ERR_WORKSPACE = 4,   /* workspace / index buffer missing or too small */
+  FQ_ERR_CUDA = 5,        /* a CUDA launch or runtime call failed */
+  FQ_ERR_TIMEOUT = 6      /* reserved: a bounded device-side wait gave up */
+} fq_status;
+
+typedef enum { FQ_F16 = 0, FQ_F32 = 1 } fq_dtype;
+
+/* Search-index kinds for fq_build_search_index. */
+typedef enum {
+  FQ_INDEX_EXACT = 0, /* conservative candidate lists: identical results to brute force */
+  FQ_INDEX_TOPC = 1   /* Cartesian grid, c codewords nearest each cell centre (approximate) */
+} fq_index_kind;
+
+/* ABI version of this header (bumped on any incompatible change). */
+int fq_abi_version(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fq_status_string(fq_status status);
+
+/* d' = k * ceil(d / k), or 0 when (d, k) is unsupported. */
+int fq_padded_dim(int d, int k);
+
+/* P, the payload bytes of one record (summary sec. 2.3: b = log2(N)/k bits per coordinate,
+ * so m * log2(N) bits per vector), or 0 when (d, k, N) is unsupported. */
+size_t fq_payload_bytes(int d, int k, int N);
+
+/*
+ * fq_encode - the FibQuant encoder (summary sec. 2.3 "encoder").
+ *   x          [n, d] row-major, fp16 or fp32 (x_type); any 2-byte (fp16) / 4-byte (fp32)
+ *              aligned address.
+ *   rot        [d', d'] fp32 Haar rotation.       codebook  [N, k] fp32.
+ *   codes      [n, P] bytes (output), any address.  norms [n] fp16 bits (output), 2-byte aligned.
+ *   search_index  NULL for brute force over all N codewords, or a device copy of a buffer
+ *              made by fq_build_search_index for this exact codebook, d and k (8-byte aligned).
+ * A zero vector encodes as norm +0 with all indices 0.  Ties between codewords resolve to
+ * the lowest index.  FQ_INDEX_EXACT gives the brute-force result; FQ_INDEX_TOPC may not.
+ */
+fq_status fq_encode(const void* x, fq_dtype x_type, int64_t n, int d, int k, int N,
+                    const float* rot, const float* codebook, uint8_t* codes, uint16_t* norms,
+                    const void* search_index, void* stream);
+
+/*
+ * fq_decode - the FibQuant decoder (summary sec. 2.3 "decoder"): y_t = nu_t (Pi^T zhat_t)[0:d]
+ * with zhat_t the concatenated codewords of record t.
+ *   codes [n, P], norms [n] as produced by fq_encode (norms 2-byte aligned).
+ *   y     [n, d] output, fp32 or fp16 (y_type, fp16 is round-to-nearest-even of the fp32
+ *         result); 4-byte (fp32) or 2-byte (fp16) aligned.
+ * Random access: to decode tokens [t0, t0 + n) pass codes + t0 * P and norms + t0.
+ */
+fq_status fq_decode(const uint8_t* codes, const uint16_t* norms, int64_t n, int d, int k, int N,
+                    const float* rot, const float* codebook, void* y, fq_dtype y_type,
+                    void* stream);
+
+/*
+ * Workspace bytes fq_attn_decode needs for these sizes (the split-softmax partials), or 0
+ * when the sizes are unsupported.  The value depends only on the arguments.
+ */
+size_t fq_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int d, int kV);
+
+/*
+ * fq_attn_decode - one decode-attention step over a FibQuant-compressed KV cache:
+ *   out[b, h] = sum_t softmax_t(scale * q[b,h] . khat[b,g,t]) vhat[b,g,t],  g = h / (Hq/Hkv),
+ * computed without decompressing: q is rotated once by Pi_K, scores come from per-block
+ * dot-product tables LUT[j][c] = (Pi_K q)_j . C_K[c] times the key norm, values are
+ * accumulated in the rotated domain and rotated back by Pi_V^T once per head.
+ *   q        [B, Hq, d] fp16 bits.         out [B, Hq, d] fp32.
+ *   k_codes  [B, Hkv, T, P_K] bytes;  k_norms [B, Hkv, T] fp16 bits (kK, NK, rotK, cbK).
+ *   v_codes  [B, Hkv, T, P_V] bytes;  v_norms [B, Hkv, T] fp16 bits (kV, NV, rotV, cbV).
+ *   workspace  device buffer of at least fq_attn_workspace_bytes(...) bytes, 16-byte aligned,
+ *              owned by the caller, overwritten by the call (no state survives it).
+ * Requires Hkv >= 1, Hq % Hkv == 0, Hq / Hkv <= 16, T >= 1, d <= 128, N_K, N_V <= 1024.
+ */
+fq_status fq_attn_decode(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int d,
+                         const uint8_t* k_codes, const uint16_t* k_norms, int kK, int NK,
+                         const float* rotK, const float* cbK,
+                         const uint8_t* v_codes, const uint16_t* v_norms, int kV, int NV,
+                         const float* rotV, const float* cbV,
+                         float scale, float* out, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * fq_build_search_index - builds, on the HOST, the candidate table fq_encode can use instead
+ * of brute force (Block Sphere VQ notes, key design 2, "Cartesian LUT": a grid of L cells per
+ * axis over the block space, each cell holding a short candidate list).
+ *   codebook_host  [N, k] fp32 host array (the same values later passed to fq_encode).
+ *   d              vector length the index will be used with (sets the grid range).
+ *   kind           FQ_INDEX_EXACT: every codeword that can be nearest to some point of the
+ *                  cell is listed (so the search equals brute force); c is ignored.
+ *                  FQ_INDEX_TOPC: the c codewords nearest to each cell centre (approximate).
+ *   L              cells per axis (2..256; L^k <= 2^22).
+ *   index_host     host output buffer of index_capacity bytes, or NULL to query the size.
+ *   index_bytes    (host, out) the exact size the index needs.
+ * Returns FQ_ERR_WORKSPACE (with *index_bytes set) when index_host is NULL or too small.
+ * The caller copies the buffer to device memory (8-byte aligned) and passes it to fq_encode.
+ */
+fq_status fq_build_search_index(const float* codebook_host, int d, int k, int N, int kind,
+                                int L, int c, void* index_host, size_t index_capacity,
+                                size_t* index_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FQ_H_ */

@@ -1,0 +1,10 @@
+"""FibQuant KV-cache codec for NVIDIA B200 (sm_100a).
+
+The compute path is libfq.so (hand-written CUDA behind the C ABI of include/fq.h); this package
+holds its thin ctypes binding (``_lib``), the table loader (``tables``), the seeded synthetic
+workloads (``workloads``) and the in-tree build step (``build``).  Importing the package does
+not load the library; the first compute call does, and raises if it is missing.
+"""
+from ._lib import (FQ_F16, FQ_F32, FQ_INDEX_EXACT, FQ_INDEX_TOPC, FQError,  # noqa: F401
+                   fq_attn_decode, fq_attn_workspace_bytes, fq_build_search_index, fq_decode,
+                   fq_encode, fq_padded_dim, fq_payload_bytes, lib, status_string)

@@ -1,0 +1,187 @@
+"""ctypes binding of libfq (the C ABI in include/fq.h): argument marshalling only.
+
+Every function here checks tensor shapes/dtypes/devices, passes ``data_ptr()`` values and the
+current CUDA stream to the C entry point of the same name, and raises FQError on a non-OK
+status.  All computation happens in the CUDA kernels of libfq.so; there is no fallback: if the
+library is missing, importing a compute function raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfq.so")
+
+FQ_F16 = 0
+FQ_F32 = 1
+FQ_INDEX_EXACT = 0
+FQ_INDEX_TOPC = 1
+
+_c_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+_i = ctypes.c_int
+
+_SIGS = {
+    "fq_abi_version": (_i, []),
+    "fq_status_string": (ctypes.c_char_p, [_i]),
+    "fq_padded_dim": (_i, [_i, _i]),
+    "fq_payload_bytes": (_sz, [_i, _i, _i]),
+    "fq_encode": (_i, [_vp, _i, _c_i64, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fq_decode": (_i, [_vp, _vp, _c_i64, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
+    "fq_attn_workspace_bytes": (_sz, [_i, _i, _i, _c_i64, _i, _i]),
+    "fq_attn_decode": (_i, [_vp, _i, _i, _i, _c_i64, _i,
+                            _vp, _vp, _i, _i, _vp, _vp,
+                            _vp, _vp, _i, _i, _vp, _vp,
+                            ctypes.c_float, _vp, _vp, _sz, _vp]),
+    "fq_build_search_index": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _sz,
+                                   ctypes.POINTER(_sz)]),
+}
+
+_lib = None
+
+
+class FQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: status {status} ({status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libfq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m random_access_kv_fq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIGS)
+
+
+def status_string(status: int) -> str:
+    return lib().fq_status_string(int(status)).decode()
+
+
+def _check(fn: str, st: int) -> None:
+    if st != 0:
+        raise FQError(fn, st)
+
+
+def fq_padded_dim(d: int, k: int) -> int:
+    return int(lib().fq_padded_dim(d, k))
+
+
+def fq_payload_bytes(d: int, k: int, N: int) -> int:
+    return int(lib().fq_payload_bytes(d, k, N))
+
+
+def fq_attn_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, d: int, kV: int) -> int:
+    return int(lib().fq_attn_workspace_bytes(B, Hq, Hkv, T, d, kV))
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return FQ_F16
+    if t.dtype == torch.float32:
+        return FQ_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def fq_encode(x, rot, codebook, k: int, N: int, codes=None, norms=None, search_index=None,
+              stream=None):
+    """Encode rows of x [n, d] (fp16/fp32, CUDA).  Returns (codes uint8 [n, P], norms int16
+    [n] holding fp16 bit patterns; view them with .view(torch.float16))."""
+    import torch
+    assert x.dim() == 2 and x.is_cuda and x.is_contiguous()
+    n, d = x.shape
+    P = fq_payload_bytes(d, k, N)
+    if codes is None:
+        codes = torch.empty((n, max(P, 1)), dtype=torch.uint8, device=x.device)
+    if norms is None:
+        norms = torch.empty((n,), dtype=torch.int16, device=x.device)
+    st = lib().fq_encode(_ptr(x), _dtype_code(x), n, d, k, N, _ptr(rot), _ptr(codebook),
+                         _ptr(codes), _ptr(norms), _ptr(search_index), _stream(stream))
+    _check("fq_encode", st)
+    return codes, norms
+
+
+def fq_decode(codes, norms, rot, codebook, d: int, k: int, N: int, out_dtype=None, y=None,
+              stream=None):
+    """Decode n records into y [n, d] (fp32 by default, or fp16)."""
+    import torch
+    n = codes.shape[0]
+    if y is None:
+        y = torch.empty((n, d), dtype=out_dtype or torch.float32, device=codes.device)
+    st = lib().fq_decode(_ptr(codes), _ptr(norms), n, d, k, N, _ptr(rot), _ptr(codebook),
+                         _ptr(y), _dtype_code(y), _stream(stream))
+    _check("fq_decode", st)
+    return y
+
+
+def fq_attn_decode(q, k_codes, k_norms, kK: int, NK: int, rotK, cbK, v_codes, v_norms,
+                   kV: int, NV: int, rotV, cbV, scale: Optional[float] = None, out=None,
+                   workspace=None, stream=None):
+    """One decode-attention step.  q [B, Hq, d] fp16; k/v codes [B, Hkv, T, P]; norms
+    [B, Hkv, T] (fp16 bits).  Returns out [B, Hq, d] fp32."""
+    import torch
+    B, Hq, d = q.shape
+    _, Hkv, T, _ = k_codes.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    need = fq_attn_workspace_bytes(B, Hq, Hkv, T, d, kV)
+    if workspace is None and need > 0:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().fq_attn_decode(_ptr(q), B, Hq, Hkv, T, d,
+                              _ptr(k_codes), _ptr(k_norms), kK, NK, _ptr(rotK), _ptr(cbK),
+                              _ptr(v_codes), _ptr(v_norms), kV, NV, _ptr(rotV), _ptr(cbV),
+                              float(scale), _ptr(out), _ptr(workspace), ws_bytes,
+                              _stream(stream))
+    _check("fq_attn_decode", st)
+    return out
+
+
+def fq_build_search_index(codebook, d: int, k: int, N: int, kind: int, L: int,
+                          c: int) -> np.ndarray:
+    """Build the grid candidate index on the host; returns a uint8 numpy buffer to upload."""
+    cb = np.ascontiguousarray(np.asarray(codebook, dtype=np.float32))
+    need = _sz(0)
+    st = lib().fq_build_search_index(cb.ctypes.data, d, k, N, kind, L, c, None, 0,
+                                     ctypes.byref(need))
+    if st not in (0, 4):
+        _check("fq_build_search_index", st)
+    buf = np.zeros(int(need.value), dtype=np.uint8)
+    st = lib().fq_build_search_index(cb.ctypes.data, d, k, N, kind, L, c, buf.ctypes.data,
+                                     buf.size, ctypes.byref(need))
+    _check("fq_build_search_index", st)
+    return buf

@@ -1,0 +1,166 @@
+// extern "C" entry points of libfq: argument validation and dispatch.  No entry point
+// allocates device memory, synchronises the stream, or keeps state between calls.
+#include <cmath>
+#include <cstdint>
+
+#include "fq_internal.h"
+#include "codec_sm100.h"
+
+namespace fq {
+
+fq_status make_shape(int d, int k, int N, Shape* s) {
+  if (d < 1 || d > kMaxD || k < 1 || k > kMaxK || k > d) return FQ_ERR_UNSUPPORTED;
+  if (N < 2 || N > kMaxN || (N & (N - 1)) != 0) return FQ_ERR_UNSUPPORTED;
+  int B = 0;
+  while ((1 << B) < N) ++B;
+  s->d = d;
+  s->k = k;
+  s->N = N;
+  s->dp = k * ((d + k - 1) / k);
+  s->m = s->dp / k;
+  s->B = B;
+  s->P = (s->m * B + 7) / 8;
+  return FQ_OK;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static fq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FQ_OK : FQ_ERR_CUDA; }
+
+}  // namespace fq
+
+using namespace fq;
+
+extern "C" {
+
+int fq_abi_version(void) { return 1; }
+
+const char* fq_status_string(fq_status st) {
+  switch (st) {
+    case FQ_OK: return "ok";
+    case FQ_ERR_INVALID_ARG: return "invalid argument";
+    case FQ_ERR_UNSUPPORTED: return "unsupported size";
+    case FQ_ERR_ALIGNMENT: return "misaligned pointer";
+    case FQ_ERR_WORKSPACE: return "workspace or index buffer missing or too small";
+    case FQ_ERR_CUDA: return "CUDA error";
+    case FQ_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+int fq_padded_dim(int d, int k) {
+  Shape s;
+  if (make_shape(d, k, 2, &s) != FQ_OK) return 0;
+  return s.dp;
+}
+
+size_t fq_payload_bytes(int d, int k, int N) {
+  Shape s;
+  if (make_shape(d, k, N, &s) != FQ_OK) return 0;
+  return (size_t)s.P;
+}
+
+fq_status fq_encode(const void* x, fq_dtype x_type, int64_t n, int d, int k, int N,
+                    const float* rot, const float* codebook, uint8_t* codes, uint16_t* norms,
+                    const void* search_index, void* stream) {
+  Shape s;
+  fq_status st = make_shape(d, k, N, &s);
+  if (st != FQ_OK) return st;
+  if (n < 0 || (x_type != FQ_F16 && x_type != FQ_F32)) return FQ_ERR_INVALID_ARG;
+  if (n == 0) return FQ_OK;
+  if (!x || !rot || !codebook || !codes || !norms) return FQ_ERR_INVALID_ARG;
+  if (!aligned(x, x_type == FQ_F16 ? 2 : 4) || !aligned(norms, 2) || !aligned(rot, 4) ||
+      !aligned(codebook, 4) || (search_index && !aligned(search_index, 8)))
+    return FQ_ERR_ALIGNMENT;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (sm100::encode_supported(x_type, s, x, codes, norms))
+    return from_cuda(sm100::launch_encode(x, x_type, n, s, rot, codebook, codes, norms,
+                                          search_index, cs));
+  return from_cuda(launch_encode_generic(x, x_type, n, s, rot, codebook, codes, norms,
+                                         search_index, cs));
+}
+
+fq_status fq_decode(const uint8_t* codes, const uint16_t* norms, int64_t n, int d, int k, int N,
+                    const float* rot, const float* codebook, void* y, fq_dtype y_type,
+                    void* stream) {
+  Shape s;
+  fq_status st = make_shape(d, k, N, &s);
+  if (st != FQ_OK) return st;
+  if (n < 0 || (y_type != FQ_F16 && y_type != FQ_F32)) return FQ_ERR_INVALID_ARG;
+  if (n == 0) return FQ_OK;
+  if (!codes || !norms || !rot || !codebook || !y) return FQ_ERR_INVALID_ARG;
+  if (!aligned(norms, 2) || !aligned(rot, 4) || !aligned(codebook, 4) ||
+      !aligned(y, y_type == FQ_F16 ? 2 : 4))
+    return FQ_ERR_ALIGNMENT;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (sm100::decode_supported(y_type, s, codes, norms, y))
+    return from_cuda(sm100::launch_decode(codes, norms, n, s, rot, codebook, y, y_type, cs));
+  return from_cuda(launch_decode_generic(codes, norms, n, s, rot, codebook, y, y_type, cs));
+}
+
+static fq_status attn_shapes(int B, int Hq, int Hkv, int64_t T, int d, int kK, int NK, int kV,
+                             int NV, Shape* ks, Shape* vs) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || T < 0 || Hq % Hkv != 0) return FQ_ERR_INVALID_ARG;
+  if (Hq / Hkv > 16 || d > 128) return FQ_ERR_UNSUPPORTED;
+  fq_status st = make_shape(d, kK, NK, ks);
+  if (st != FQ_OK) return st;
+  st = make_shape(d, kV, NV, vs);
+  if (st != FQ_OK) return st;
+  if (NK > 1024 || NV > 1024) return FQ_ERR_UNSUPPORTED;
+  return FQ_OK;
+}
+
+size_t fq_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int d, int kV) {
+  Shape ks, vs;
+  if (attn_shapes(B, Hq, Hkv, T, d, 1, 2, kV, 2, &ks, &vs) != FQ_OK) return 0;
+  if (T == 0) return 0;
+  int splits = attn_splits(B, Hkv, T);
+  return attn_partials_bytes(B, Hq, splits, vs.dp);
+}
+
+fq_status fq_attn_decode(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int d,
+                         const uint8_t* k_codes, const uint16_t* k_norms, int kK, int NK,
+                         const float* rotK, const float* cbK, const uint8_t* v_codes,
+                         const uint16_t* v_norms, int kV, int NV, const float* rotV,
+                         const float* cbV, float scale, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  AttnArgs a;
+  fq_status st = attn_shapes(B, Hq, Hkv, T, d, kK, NK, kV, NV, &a.ks, &a.vs);
+  if (st != FQ_OK) return st;
+  if (!std::isfinite(scale)) return FQ_ERR_INVALID_ARG;
+  if (!q || !out) return FQ_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (T == 0)
+    return from_cuda(cudaMemsetAsync(out, 0, (size_t)B * Hq * d * sizeof(float), cs));
+  if (!k_codes || !k_norms || !rotK || !cbK || !v_codes || !v_norms || !rotV || !cbV)
+    return FQ_ERR_INVALID_ARG;
+  if (!aligned(q, 2) || !aligned(k_norms, 2) || !aligned(v_norms, 2) || !aligned(rotK, 4) ||
+      !aligned(cbK, 4) || !aligned(rotV, 4) || !aligned(cbV, 4) || !aligned(out, 4))
+    return FQ_ERR_ALIGNMENT;
+  a.q = q;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.T = T;
+  a.d = d;
+  a.k_codes = k_codes;
+  a.k_norms = k_norms;
+  a.rotK = rotK;
+  a.cbK = cbK;
+  a.v_codes = v_codes;
+  a.v_norms = v_norms;
+  a.rotV = rotV;
+  a.cbV = cbV;
+  a.scale = scale;
+  a.out = out;
+  a.splits = attn_splits(B, Hkv, T);
+  a.tokens_per_split = attn_tokens_per_split(T, a.splits);
+  size_t need = attn_partials_bytes(B, Hq, a.splits, a.vs.dp);
+  if (!workspace || workspace_bytes < need) return FQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return FQ_ERR_ALIGNMENT;
+  a.partials = static_cast<float*>(workspace);
+  if (attn_smem_bytes(a) > 200 * 1024) return FQ_ERR_UNSUPPORTED;
+  return from_cuda(launch_attn(a, cs));
+}
+
+}  // extern "C"

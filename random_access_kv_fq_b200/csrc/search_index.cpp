@@ -1,0 +1,233 @@
+// Host-side builder of the grid candidate index used by fq_encode's pruned search.
+//
+// Block Sphere VQ notes, key design 2 ("Cartesian LUT"): split the k-dimensional block space
+// into a grid with L cells per axis, keep a short candidate list per cell, and search only
+// that list instead of all N codewords.  Two list rules:
+//   FQ_INDEX_TOPC  - the c codewords nearest to the cell centre, as the notes describe
+//                    (approximate: a block near a cell edge can have its nearest codeword
+//                    outside the list);
+//   FQ_INDEX_EXACT - every codeword that is the nearest one for some point of the (slightly
+//                    enlarged) cell, so the search returns the brute-force answer.  A codeword
+//                    n is listed when (i) its distance to the cell is at most the smallest
+//                    farthest-corner distance of any codeword (otherwise another codeword is
+//                    closer everywhere in the cell) and (ii) no other codeword is closer than
+//                    n at every point of the cell (checked exactly: the difference of squared
+//                    distances is linear, so its minimum over the box sits at a corner).
+// Grid range: [-R, R]^k with R = max |codeword coordinate| + 3 / sqrt(d'); coordinates
+// outside clamp to the edge cells, so the edge cells' boxes extend to the unit-ball bound.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "fq_internal.h"
+
+namespace fq {
+namespace {
+
+struct Grid {
+  int k, N, L, dp, n_cells;
+  double R, h;      // as defined by the rule (float64)
+  float lo_f, inv_h_f;  // what the device uses
+  double h_dev;     // cell width the device's fp32 mapping implies
+};
+
+void cell_box(const Grid& g, int flat, double* lo, double* hi) {
+  const double margin = std::max(1e-4 * g.h_dev, 1e-6);
+  for (int a = 0; a < g.k; ++a) {
+    int i = flat % g.L;
+    flat /= g.L;
+    double l = (double)g.lo_f + i * g.h_dev - margin;
+    double u = (double)g.lo_f + (i + 1) * g.h_dev + margin;
+    if (i == 0) l = std::min(l, -1.001);
+    if (i == g.L - 1) u = std::max(u, 1.001);
+    lo[a] = l;
+    hi[a] = u;
+  }
+}
+
+// Candidates of one cell under the exact rule, sorted by (distance to the box, index).
+void exact_candidates(const Grid& g, const double* C, const double* cc, int flat,
+                      std::vector<int>& out) {
+  double lo[kMaxK], hi[kMaxK];
+  cell_box(g, flat, lo, hi);
+  const int N = g.N, k = g.k;
+  std::vector<double> dmin(N);
+  double thr = INFINITY;
+  for (int n = 0; n < N; ++n) {
+    double mn = 0, mx = 0;
+    for (int a = 0; a < k; ++a) {
+      double c = C[(size_t)n * k + a];
+      double t = c < lo[a] ? lo[a] - c : (c > hi[a] ? c - hi[a] : 0.0);
+      mn += t * t;
+      double f = std::max(std::fabs(c - lo[a]), std::fabs(c - hi[a]));
+      mx += f * f;
+    }
+    dmin[n] = mn;
+    thr = std::min(thr, mx);
+  }
+  std::vector<int> cand;
+  for (int n = 0; n < N; ++n)
+    if (dmin[n] <= thr * (1.0 + 1e-12) + 1e-15) cand.push_back(n);
+  // pairwise dominance: m dominates n on the box if |p-c_n|^2 - |p-c_m|^2 > 0 for all p
+  out.clear();
+  for (int n : cand) {
+    bool dominated = false;
+    for (int mm : cand) {
+      if (mm == n) continue;
+      double f = cc[n] - cc[mm];
+      for (int a = 0; a < k; ++a) {
+        double dl = C[(size_t)mm * k + a] - C[(size_t)n * k + a];
+        f += 2.0 * std::min(lo[a] * dl, hi[a] * dl);
+      }
+      if (f > 1e-12) {
+        dominated = true;
+        break;
+      }
+    }
+    if (!dominated) out.push_back(n);
+  }
+  std::sort(out.begin(), out.end(),
+            [&](int a, int b) { return dmin[a] < dmin[b] || (dmin[a] == dmin[b] && a < b); });
+}
+
+void topc_candidates(const Grid& g, const double* C, int flat, int c, std::vector<int>& out) {
+  double centre[kMaxK];
+  for (int a = 0; a < g.k; ++a) {
+    int i = flat % g.L;
+    flat /= g.L;
+    centre[a] = -g.R + (i + 0.5) * g.h;
+  }
+  std::vector<std::pair<double, int>> dist(g.N);
+  for (int n = 0; n < g.N; ++n) {
+    double s = 0;
+    for (int a = 0; a < g.k; ++a) {
+      double t = centre[a] - C[(size_t)n * g.k + a];
+      s += t * t;
+    }
+    dist[n] = {s, n};
+  }
+  std::partial_sort(dist.begin(), dist.begin() + c, dist.end());
+  out.resize(c);
+  for (int i = 0; i < c; ++i) out[i] = dist[i].second;
+}
+
+}  // namespace
+}  // namespace fq
+
+using namespace fq;
+
+extern "C" fq_status fq_build_search_index(const float* codebook_host, int d, int k, int N,
+                                           int kind, int L, int c, void* index_host,
+                                           size_t index_capacity, size_t* index_bytes) {
+  Shape s;
+  fq_status st = make_shape(d, k, N, &s);
+  if (st != FQ_OK) return st;
+  if (!codebook_host || !index_bytes) return FQ_ERR_INVALID_ARG;
+  if (kind != FQ_INDEX_EXACT && kind != FQ_INDEX_TOPC) return FQ_ERR_INVALID_ARG;
+  if (L < 2 || L > 256) return FQ_ERR_UNSUPPORTED;
+  double cells_d = std::pow((double)L, k);
+  if (cells_d > (double)(1 << 22)) return FQ_ERR_UNSUPPORTED;
+  if (c < 1 || c > 64 || (kind == FQ_INDEX_TOPC && c > N)) return FQ_ERR_UNSUPPORTED;
+
+  Grid g;
+  g.k = k;
+  g.N = N;
+  g.L = L;
+  g.dp = s.dp;
+  g.n_cells = (int)cells_d;
+  std::vector<double> C((size_t)N * k), cc(N);
+  double maxabs = 0;
+  for (int n = 0; n < N; ++n) {
+    double sq = 0;
+    for (int a = 0; a < k; ++a) {
+      double v = codebook_host[(size_t)n * k + a];
+      if (!std::isfinite(v)) return FQ_ERR_INVALID_ARG;
+      C[(size_t)n * k + a] = v;
+      sq += v * v;
+      maxabs = std::max(maxabs, std::fabs(v));
+    }
+    cc[n] = sq;
+  }
+  g.R = maxabs + 3.0 / std::sqrt((double)s.dp);
+  g.h = 2.0 * g.R / L;
+  g.lo_f = (float)(-g.R);
+  g.inv_h_f = (float)(1.0 / g.h);
+  g.h_dev = 1.0 / (double)g.inv_h_f;
+
+  const int slots = c;
+  std::vector<std::vector<int>> lists(g.n_cells);
+  unsigned nth = std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
+  std::vector<std::thread> pool;
+  for (unsigned t = 0; t < nth; ++t) {
+    pool.emplace_back([&, t]() {
+      std::vector<int> tmp;
+      for (int f = (int)t; f < g.n_cells; f += (int)nth) {
+        if (kind == FQ_INDEX_EXACT)
+          exact_candidates(g, C.data(), cc.data(), f, tmp);
+        else
+          topc_candidates(g, C.data(), f, c, tmp);
+        lists[f] = tmp;
+      }
+    });
+  }
+  for (auto& th : pool) th.join();
+
+  const int id_bytes = ((2 * slots + 3) / 4) * 4;
+  const int entry_bytes = id_bytes + (kind == FQ_INDEX_EXACT ? 4 : 0);
+  size_t ov_elems = 0;
+  uint32_t max_cand = 0;
+  for (auto& l : lists) {
+    if (l.empty()) return FQ_ERR_INVALID_ARG;  // cannot happen: the nearest codeword survives
+    if ((int)l.size() > slots) ov_elems += 1 + (l.size() - slots);
+    max_cand = std::max<uint32_t>(max_cand, (uint32_t)l.size());
+  }
+  const size_t cells_off = sizeof(IndexHeader);
+  size_t ov_off = cells_off + (size_t)g.n_cells * entry_bytes;
+  ov_off = (ov_off + 7) & ~size_t(7);
+  size_t total = ov_off + ov_elems * 2;
+  total = (total + 7) & ~size_t(7);
+  if (total > 0xFFFFFFFFull) return FQ_ERR_UNSUPPORTED;
+  *index_bytes = total;
+  if (!index_host || index_capacity < total) return FQ_ERR_WORKSPACE;
+
+  uint8_t* out = static_cast<uint8_t*>(index_host);
+  std::memset(out, 0, total);
+  IndexHeader hdr;
+  hdr.magic = kIndexMagic;
+  hdr.version = kIndexVersion;
+  hdr.kind = kind;
+  hdr.k = k;
+  hdr.N = N;
+  hdr.L = L;
+  hdr.dp = s.dp;
+  hdr.slots = slots;
+  hdr.lo = g.lo_f;
+  hdr.inv_h = g.inv_h_f;
+  hdr.n_cells = g.n_cells;
+  hdr.entry_bytes = entry_bytes;
+  hdr.cells_offset = (uint32_t)cells_off;
+  hdr.overflow_offset = (uint32_t)ov_off;
+  hdr.overflow_elems = (uint32_t)ov_elems;
+  hdr.max_candidates = max_cand;
+  std::memcpy(out, &hdr, sizeof(hdr));
+  uint16_t* ovl = reinterpret_cast<uint16_t*>(out + ov_off);
+  size_t ov_pos = 0;
+  for (int f = 0; f < g.n_cells; ++f) {
+    const auto& l = lists[f];
+    uint8_t* e = out + cells_off + (size_t)f * entry_bytes;
+    uint16_t* ids = reinterpret_cast<uint16_t*>(e);
+    for (int i = 0; i < slots; ++i) ids[i] = (uint16_t)(i < (int)l.size() ? l[i] : l[0]);
+    if (kind == FQ_INDEX_EXACT) {
+      uint32_t w = kNoOverflow;
+      if ((int)l.size() > slots) {
+        w = (uint32_t)ov_pos;
+        ovl[ov_pos++] = (uint16_t)(l.size() - slots);
+        for (size_t i = slots; i < l.size(); ++i) ovl[ov_pos++] = (uint16_t)l[i];
+      }
+      std::memcpy(e + id_bytes, &w, 4);
+    }
+  }
+  return FQ_OK;
+}

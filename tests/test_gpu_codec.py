@@ -1,0 +1,194 @@
+"""GPU parity of fq_encode / fq_decode (through the C ABI) against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import random_access_kv_fq_b200 as fq
+from oracle import fq_oracle as fo
+from random_access_kv_fq_b200 import tables, workloads as wl
+from tests import parity as par
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _index(cb, d, rate):
+    if rate.search == "brute":
+        return None
+    kind = fq.FQ_INDEX_EXACT if rate.search == "exact" else fq.FQ_INDEX_TOPC
+    return _dev(fq.fq_build_search_index(cb, d, rate.k, rate.N, kind, rate.grid_L, rate.grid_c))
+
+
+def _oracle_encode(x, rot, cb, rate):
+    if rate.search == "top":
+        enc, bd = fo.encode_grid_topc(x, rot, cb, rate.k, rate.grid_L, rate.grid_c)
+        return enc, bd[:, :, None] if bd.ndim == 2 else bd
+    return fo.encode(x, rot, cb, rate.k), None
+
+
+def run_codec(x, rot, cb, rate, d, check_decode=True, out16=False):
+    """Encode + decode x on the GPU and check both against the oracle.  Returns the GPU
+    indices."""
+    k, N = rate.k, rate.N
+    m = fo.padded_dim(d, k) // k
+    xt, rt, ct = _dev(x), _dev(rot), _dev(cb)
+    ix = _index(cb, d, rate)
+    codes, norms = fq.fq_encode(xt, rt, ct, k, N, search_index=ix)
+    torch.cuda.synchronize()
+    gcodes, gnorms = par.to_np(codes), par.to_np(norms)
+    enc, bd = _oracle_encode(x, rot, cb, rate)
+    exempt = None
+    if bd is not None:
+        exempt = (bd.reshape(enc.idx.shape) < 1e-6)
+    gidx = par.check_records_and_indices(gcodes, enc, N, m, exempt)
+    par.check_norms(gnorms, enc)
+    if check_decode:
+        y = fq.fq_decode(codes, norms, rt, ct, d, k, N)
+        torch.cuda.synchronize()
+        ref = par.check_recon(par.to_np(y), gidx, gnorms, rot, cb, d)
+        if out16:
+            y16 = fq.fq_decode(codes, norms, rt, ct, d, k, N, out_dtype=torch.float16)
+            par.check_recon_f16(par.to_np(y16).astype(np.float64), ref)
+    return gidx
+
+
+def _table_inputs(dp, k, N, seed=wl.ROT_SEED_K):
+    return tables.rotation(dp, seed), tables.codebook(dp, k, N)
+
+
+CASES = [(w, r) for w in (wl.TOY, wl.GPT2, wl.TINYLLAMA, wl.LARGE) for r in w.rates]
+
+
+@pytest.mark.parametrize("w,rate", CASES, ids=[f"{w.name}-{r.label}" for w, r in CASES])
+def test_codec_small_slice(w, rate):
+    """Rows from every layer/head of the workload, several tiles plus a ragged tail."""
+    shape = w.cache
+    rng = np.random.default_rng(7)
+    n = 2048 + 1000 + 77 if shape.d == 64 else 1024 + 77
+    rows = np.sort(rng.choice(shape.n, size=min(n, shape.n), replace=False))
+    x = wl.rows_of(shape, rows)
+    dp = fo.padded_dim(shape.d, rate.k)
+    rot, cb = _table_inputs(dp, rate.k, rate.N)
+    run_codec(x, rot, cb, rate, shape.d, out16=True)
+
+
+@pytest.mark.parametrize("w,rate", CASES, ids=[f"{w.name}-{r.label}" for w, r in CASES])
+def test_codec_full_size_sampled(w, rate):
+    """The whole workload encoded/decoded in one call each (the launch the bench times);
+    sampled rows checked against the oracle one by one."""
+    shape = w.cache
+    dp = fo.padded_dim(shape.d, rate.k)
+    rot, cb = _table_inputs(dp, rate.k, rate.N)
+    k, N = rate.k, rate.N
+    m = dp // k
+    x = torch.empty((shape.n, shape.d), dtype=torch.float16 if shape.dtype == "f16" else torch.float32,
+                    device="cuda")
+    for row, s in wl.slabs(shape):
+        x[row:row + s.shape[0]].copy_(torch.from_numpy(s))
+    rt, ct = _dev(rot), _dev(cb)
+    ix = _index(cb, shape.d, rate)
+    codes, norms = fq.fq_encode(x, rt, ct, k, N, search_index=ix)
+    y = fq.fq_decode(codes, norms, rt, ct, shape.d, k, N)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(11)
+    sample = np.sort(rng.choice(shape.n, size=min(4096, shape.n), replace=False))
+    sample = np.unique(np.concatenate([sample, [0, shape.n - 1]]))
+    st = torch.from_numpy(sample).cuda()
+    xs = wl.rows_of(shape, sample)
+    np.testing.assert_array_equal(par.to_np(x[st]), xs)
+    gcodes = par.to_np(codes[st])
+    gnorms = par.to_np(norms[st])
+    enc, bd = _oracle_encode(xs, rot, cb, rate)
+    exempt = None if bd is None else (bd.reshape(enc.idx.shape) < 1e-6)
+    gidx = par.check_records_and_indices(gcodes, enc, N, m, exempt)
+    par.check_norms(gnorms, enc)
+    par.check_recon(par.to_np(y[st]), gidx, gnorms, rot, cb, shape.d)
+
+
+# ------------------------------------------------------------------ edge cases
+
+def test_empty_and_single():
+    rot, cb = _table_inputs(64, 2, 16)
+    x = torch.empty((0, 64), dtype=torch.float16, device="cuda")
+    codes, norms = fq.fq_encode(x, _dev(rot), _dev(cb), 2, 16)
+    assert codes.shape[0] == 0
+    x1 = wl.gaussian_rows(1, 64, 3)
+    run_codec(x1, rot, cb, wl.Rate(2, 16), 64)
+
+
+def test_zero_vectors_and_extremes():
+    rot, cb = _table_inputs(64, 2, 16)
+    x = wl.gaussian_rows(300, 64, 4)
+    x[5] = 0
+    x[17] = 0
+    x[40] = np.float16(65504.0)       # largest fp16: norm overflows fp16 -> inf
+    x[41] = np.float16(6e-8)          # subnormal inputs
+    x[42, 3] = np.float16(-1.0)
+    x[42, :3] = 0
+    x[42, 4:] = 0                     # a one-hot vector
+    run_codec(x, rot, cb, wl.Rate(2, 16), 64, check_decode=False)
+    xs = np.delete(x, [40], axis=0)   # decode check without the inf-norm row
+    run_codec(xs, rot, cb, wl.Rate(2, 16), 64)
+
+
+def test_codeword_aligned_inputs_reproduce_indices():
+    """'Shell' codebooks c_n = u_n / sqrt(m) make every concatenation of codewords a unit
+    vector, so x = nu Pi^T zhat has every block exactly on a codeword: the GPU must return
+    exactly the constructed indices and decode x back to fp32 accuracy."""
+    import math
+    for d, k, N in ((64, 2, 16), (64, 4, 8), (64, 2, 256), (128, 4, 64)):
+        m = d // k
+        rot = tables.rotation(d, 17)
+        cb = (fo.init_directions(k, N) / math.sqrt(m)).astype(np.float32)
+        rng = np.random.default_rng(d + k + N)
+        idx = rng.integers(0, N, size=(500, m))
+        zhat = cb.astype(np.float64)[idx].reshape(500, d)
+        x = (8.0 * (zhat @ rot.astype(np.float64))).astype(np.float32)
+        gidx = run_codec(x, rot, cb, wl.Rate(k, N), d)
+        np.testing.assert_array_equal(gidx, idx)
+
+
+@pytest.mark.parametrize("d,k,N,dtype", [(64, 1, 4, np.float16), (64, 1, 16, np.float32),
+                                         (256, 2, 16, np.float16), (128, 2, 16, np.float16),
+                                         (96, 5, 32, np.float32), (17, 3, 8, np.float32),
+                                         (32, 4, 65536, np.float16), (128, 8, 256, np.float16),
+                                         (64, 2, 2, np.float16)])
+def test_other_shapes(d, k, N, dtype):
+    """Shapes outside the workloads (scalar k = 1, k not dividing d, d = 256, N = 65536)."""
+    dp = fo.padded_dim(d, k)
+    rot = fo.haar_rotation(dp, 99).astype(np.float32)
+    cb = fo.init_codebook(dp, k, N).astype(np.float32) if k > 1 else \
+        np.sort(fo.scalar_lloyd(dp, N)).astype(np.float32)[:, None]
+    n = 200 if N < 65536 else 40
+    x = wl.gaussian_rows(n, d, d * 7 + k, dtype=dtype)
+    run_codec(x, rot, cb, wl.Rate(k, N), d, out16=True)
+
+
+def test_random_access_decode_at_unaligned_offsets():
+    """Decoding any token range from codes + t0 * P (P = 17: odd byte offsets) gives the same
+    values as decoding the whole cache."""
+    rot, cb = _table_inputs(66, 3, 64)
+    x = wl.gaussian_rows(1000, 64, 8)
+    rt, ct = _dev(rot), _dev(cb)
+    codes, norms = fq.fq_encode(_dev(x), rt, ct, 3, 64)
+    full = fq.fq_decode(codes, norms, rt, ct, 64, 3, 64)
+    flat = codes.reshape(-1)
+    for t0, cnt in ((1, 5), (333, 100), (999, 1), (7, 993)):
+        sub = flat[t0 * 17:(t0 + cnt) * 17].reshape(cnt, 17)
+        y = fq.fq_decode(sub, norms[t0:t0 + cnt], rt, ct, 64, 3, 64)
+        torch.testing.assert_close(y, full[t0:t0 + cnt], rtol=0, atol=0)
+
+
+def test_index_with_wrong_codebook_falls_back_to_exact_search():
+    """An index built for another (k, N) is ignored (the result is the brute-force one)."""
+    rot, cb = _table_inputs(64, 2, 16)
+    _, cb8 = _table_inputs(64, 2, 8)
+    ix = _dev(fq.fq_build_search_index(cb8, 64, 2, 8, fq.FQ_INDEX_EXACT, 32, 2))
+    x = wl.gaussian_rows(500, 64, 9)
+    rt, ct = _dev(rot), _dev(cb)
+    c1, n1 = fq.fq_encode(_dev(x), rt, ct, 2, 16, search_index=ix)
+    c2, n2 = fq.fq_encode(_dev(x), rt, ct, 2, 16)
+    assert torch.equal(c1, c2) and torch.equal(n1, n2)
