@@ -48,9 +48,8 @@ __device__ __forceinline__ int index_nearest(const float* zb, int k, const float
     stride *= h->L;
   }
   const uint8_t* entry = index + h->cells_offset + (size_t)flat * h->entry_bytes;
-  const uint16_t* ids = reinterpret_cast<const uint16_t*>(entry);
   uint32_t ov = kNoOverflow;
-  if (h->kind == FQ_INDEX_EXACT)
+  if (index_has_overflow(*h))
     ov = *reinterpret_cast<const uint32_t*>(entry + h->entry_bytes - 4);
   const uint16_t* ovl = reinterpret_cast<const uint16_t*>(index + h->overflow_offset);
   int n_extra = (ov == kNoOverflow) ? 0 : ovl[ov];
@@ -58,7 +57,7 @@ __device__ __forceinline__ int index_nearest(const float* zb, int k, const float
   float best = INFINITY;
   int bi = 0x7fffffff;
   for (int i = lane; i < total; i += 32) {
-    int c = (i < h->slots) ? ids[i] : ovl[ov + 1 + (i - h->slots)];
+    int c = (i < h->slots) ? index_entry_id(entry, i, h->id_bytes) : ovl[ov + 1 + (i - h->slots)];
     float dist = 0.f;
     for (int r = 0; r < k; ++r) {
       float t = zb[r] - __ldg(cb + (size_t)c * k + r);

@@ -26,13 +26,19 @@ struct Shape {
 fq_status make_shape(int d, int k, int N, Shape* s);
 
 // ---- search index (host builder and device view) ------------------------------------------
-// Layout of the buffer made by fq_build_search_index (all little-endian, 8-byte aligned):
+// Layout of the buffer made by fq_build_search_index (little-endian, 8-byte aligned):
 //   IndexHeader (64 bytes)
-//   cells:    n_cells entries of `entry_bytes` bytes each; an entry is `slots` uint16 candidate
-//             ids followed (when entry_bytes > 2*slots) by padding and a uint32 overflow word;
-//             ids of a cell with fewer candidates than slots are padded by repeating the first.
+//   cells:    n_cells entries of `entry_bytes` bytes.  An entry holds `slots` candidate ids of
+//             `id_bytes` bytes each (1 when N <= 256, else 2), sorted by increasing index; the
+//             rest of the id area (up to a 4-byte boundary) repeats the last inline id; when max_candidates > slots (exact kind only)
+//             the entry ends with a uint32 overflow word.
 //   overflow: uint16 array; an overflow word w != 0xFFFFFFFF points at element w, which holds
-//             the number of extra candidates followed by their ids.
+//             the number of further candidates followed by their ids (all larger than the
+//             inline ones).
+// Cell of a block z (k coordinates): c_a = clamp(floor((z_a - lo) * inv_h), 0, L - 1),
+// flat = sum_a c_a L^a.  Every list is built for the cell enlarged by a margin, so the fp32
+// rounding of this mapping cannot move a block to a cell whose list misses its nearest
+// codeword (exact kind).
 struct IndexHeader {
   uint32_t magic;        // kIndexMagic
   uint32_t version;      // kIndexVersion
@@ -47,12 +53,20 @@ struct IndexHeader {
   uint32_t cells_offset; // byte offset of the cell table
   uint32_t overflow_offset;
   uint32_t overflow_elems;
-  uint32_t max_candidates;  // longest candidate list (inline + overflow)
+  uint16_t max_candidates;  // longest candidate list
+  uint16_t id_bytes;        // 1 or 2
 };
 static_assert(sizeof(IndexHeader) == 64, "index header is 64 bytes");
 constexpr uint32_t kIndexMagic = 0x58495146u;  // "FQIX"
-constexpr uint32_t kIndexVersion = 1;
+constexpr uint32_t kIndexVersion = 2;
 constexpr uint32_t kNoOverflow = 0xFFFFFFFFu;
+
+__host__ __device__ inline bool index_has_overflow(const IndexHeader& h) {
+  return h.kind == FQ_INDEX_EXACT && h.max_candidates > h.slots;
+}
+__host__ __device__ inline int index_entry_id(const uint8_t* entry, int i, int id_bytes) {
+  return id_bytes == 1 ? entry[i] : reinterpret_cast<const uint16_t*>(entry)[i];
+}
 
 // ---- launchers (return cudaGetLastError() of the launch) ----------------------------------
 cudaError_t launch_encode_generic(const void* x, fq_dtype xt, int64_t n, const Shape& s,

@@ -34,7 +34,7 @@ struct Grid {
 };
 
 void cell_box(const Grid& g, int flat, double* lo, double* hi) {
-  const double margin = std::max(1e-4 * g.h_dev, 1e-6);
+  const double margin = 1e-3 * g.h_dev + 1e-6;
   for (int a = 0; a < g.k; ++a) {
     int i = flat % g.L;
     flat /= g.L;
@@ -88,8 +88,7 @@ void exact_candidates(const Grid& g, const double* C, const double* cc, int flat
     }
     if (!dominated) out.push_back(n);
   }
-  std::sort(out.begin(), out.end(),
-            [&](int a, int b) { return dmin[a] < dmin[b] || (dmin[a] == dmin[b] && a < b); });
+  std::sort(out.begin(), out.end());  // by index: a strict-less scan keeps the lowest on ties
 }
 
 void topc_candidates(const Grid& g, const double* C, int flat, int c, std::vector<int>& out) {
@@ -111,6 +110,7 @@ void topc_candidates(const Grid& g, const double* C, int flat, int c, std::vecto
   std::partial_sort(dist.begin(), dist.begin() + c, dist.end());
   out.resize(c);
   for (int i = 0; i < c; ++i) out[i] = dist[i].second;
+  std::sort(out.begin(), out.end());
 }
 
 }  // namespace
@@ -174,8 +174,7 @@ extern "C" fq_status fq_build_search_index(const float* codebook_host, int d, in
   }
   for (auto& th : pool) th.join();
 
-  const int id_bytes = ((2 * slots + 3) / 4) * 4;
-  const int entry_bytes = id_bytes + (kind == FQ_INDEX_EXACT ? 4 : 0);
+  const int id_bytes = N <= 256 ? 1 : 2;
   size_t ov_elems = 0;
   uint32_t max_cand = 0;
   for (auto& l : lists) {
@@ -183,6 +182,10 @@ extern "C" fq_status fq_build_search_index(const float* codebook_host, int d, in
     if ((int)l.size() > slots) ov_elems += 1 + (l.size() - slots);
     max_cand = std::max<uint32_t>(max_cand, (uint32_t)l.size());
   }
+  if (max_cand > 65535) return FQ_ERR_UNSUPPORTED;
+  const bool overflow = kind == FQ_INDEX_EXACT && (int)max_cand > slots;
+  const int ids_bytes = ((slots * id_bytes + 3) / 4) * 4;
+  const int entry_bytes = ids_bytes + (overflow ? 4 : 0);
   const size_t cells_off = sizeof(IndexHeader);
   size_t ov_off = cells_off + (size_t)g.n_cells * entry_bytes;
   ov_off = (ov_off + 7) & ~size_t(7);
@@ -210,23 +213,30 @@ extern "C" fq_status fq_build_search_index(const float* codebook_host, int d, in
   hdr.cells_offset = (uint32_t)cells_off;
   hdr.overflow_offset = (uint32_t)ov_off;
   hdr.overflow_elems = (uint32_t)ov_elems;
-  hdr.max_candidates = max_cand;
+  hdr.max_candidates = (uint16_t)max_cand;
+  hdr.id_bytes = (uint16_t)id_bytes;
   std::memcpy(out, &hdr, sizeof(hdr));
   uint16_t* ovl = reinterpret_cast<uint16_t*>(out + ov_off);
   size_t ov_pos = 0;
   for (int f = 0; f < g.n_cells; ++f) {
     const auto& l = lists[f];
     uint8_t* e = out + cells_off + (size_t)f * entry_bytes;
-    uint16_t* ids = reinterpret_cast<uint16_t*>(e);
-    for (int i = 0; i < slots; ++i) ids[i] = (uint16_t)(i < (int)l.size() ? l[i] : l[0]);
-    if (kind == FQ_INDEX_EXACT) {
+    const int pad_slots = ids_bytes / id_bytes;  // pad the whole id area with the last id
+    for (int i = 0; i < pad_slots; ++i) {
+      int id = l[std::min<int>(std::min(i, slots - 1), (int)l.size() - 1)];
+      if (id_bytes == 1)
+        e[i] = (uint8_t)id;
+      else
+        reinterpret_cast<uint16_t*>(e)[i] = (uint16_t)id;
+    }
+    if (overflow) {
       uint32_t w = kNoOverflow;
       if ((int)l.size() > slots) {
         w = (uint32_t)ov_pos;
         ovl[ov_pos++] = (uint16_t)(l.size() - slots);
         for (size_t i = slots; i < l.size(); ++i) ovl[ov_pos++] = (uint16_t)l[i];
       }
-      std::memcpy(e + id_bytes, &w, 4);
+      std::memcpy(e + ids_bytes, &w, 4);
     }
   }
   return FQ_OK;

@@ -106,14 +106,14 @@ GPT2 = CodecWorkload(
     "gpt2small_12Lx12Hx1024T_d64",
     CacheShape(batch=1, layers=12, heads=12, tokens=1024, d=64, sigma=1.0, outliers=True,
                dtype="f16", seed=1002),
-    (Rate(3, 64, "exact", grid_L=16, grid_c=4), Rate(4, 8, "brute")),
+    (Rate(3, 64, "exact", grid_L=16, grid_c=10), Rate(4, 8, "brute")),
 )
 TINYLLAMA = CodecWorkload(
     "tinyllama_22Lx4Hx2048Tx8B_d64",
     CacheShape(batch=8, layers=22, heads=4, tokens=2048, d=64, sigma=1.0, outliers=True,
                dtype="f16", seed=1003),
-    (Rate(2, 256, "exact", grid_L=128, grid_c=4), Rate(2, 16, "exact", grid_L=64, grid_c=2),
-     Rate(2, 8, "exact", grid_L=32, grid_c=2)),
+    (Rate(2, 256, "exact", grid_L=128, grid_c=4), Rate(2, 16, "exact", grid_L=64, grid_c=3),
+     Rate(2, 8, "exact", grid_L=32, grid_c=3)),
 )
 LARGE = CodecWorkload(
     "large_32Lx8Hx32768T_d128",

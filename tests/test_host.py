@@ -111,21 +111,28 @@ def _parse_index(buf):
     h = np.frombuffer(buf[:64].tobytes(), dtype=np.int32)
     f = np.frombuffer(buf[:64].tobytes(), dtype=np.float32)
     u = np.frombuffer(buf[:64].tobytes(), dtype=np.uint32)
+    u16 = np.frombuffer(buf[:64].tobytes(), dtype=np.uint16)
     hdr = dict(kind=h[2], k=h[3], N=h[4], L=h[5], dp=h[6], slots=h[7], lo=f[8], inv_h=f[9],
-               n_cells=h[10], entry_bytes=h[11], cells_offset=u[12], overflow_offset=u[13])
-    assert u[0] == 0x58495146
+               n_cells=h[10], entry_bytes=h[11], cells_offset=u[12], overflow_offset=u[13],
+               max_candidates=int(u16[30]), id_bytes=int(u16[31]))
+    assert u[0] == 0x58495146 and u[1] == 2
     return hdr
 
 
-def _cell_list(buf, hdr, cell):
+def _cell_ids(buf, hdr, cell):
     e = buf[hdr["cells_offset"] + cell * hdr["entry_bytes"]:][:hdr["entry_bytes"]]
-    ids = list(np.frombuffer(e[:2 * hdr["slots"]].tobytes(), dtype=np.uint16))
-    if hdr["kind"] == 0:
+    dt = np.uint8 if hdr["id_bytes"] == 1 else np.uint16
+    ids = [int(i) for i in np.frombuffer(e[:hdr["slots"] * hdr["id_bytes"]].tobytes(), dtype=dt)]
+    if hdr["kind"] == 0 and hdr["max_candidates"] > hdr["slots"]:
         w = int(np.frombuffer(e[-4:].tobytes(), dtype=np.uint32)[0])
         if w != 0xFFFFFFFF:
             ov = np.frombuffer(buf[hdr["overflow_offset"]:].tobytes(), dtype=np.uint16)
-            ids += list(ov[w + 1:w + 1 + ov[w]])
-    return set(int(i) for i in ids)
+            ids += [int(i) for i in ov[w + 1:w + 1 + ov[w]]]
+    return ids
+
+
+def _cell_list(buf, hdr, cell):
+    return set(_cell_ids(buf, hdr, cell))
 
 
 @pytest.mark.parametrize("dp,k,N,L,slots", [(64, 2, 16, 64, 2), (64, 2, 256, 128, 4),
@@ -144,6 +151,11 @@ def test_exact_index_lists_contain_the_brute_force_nearest(dp, k, N, L, slots):
     cells = _cell_of(z, hdr)
     for zi, ci, ni in zip(z, cells, nn):
         assert int(ni) in _cell_list(buf, hdr, int(ci))
+    # lists are sorted by index (padding repeats the last id), so a strict-less scan keeps
+    # the lowest index on exact ties
+    for cell in range(0, hdr["n_cells"], max(1, hdr["n_cells"] // 500)):
+        ids = _cell_ids(buf, hdr, cell)
+        assert ids == sorted(ids)
 
 
 def test_topc_index_equals_oracle_table():
@@ -154,8 +166,7 @@ def test_topc_index_equals_oracle_table():
     R = fo.grid_range(C.astype(np.float64), 64)
     ref = fo.grid_topc_table(C.astype(np.float64), R, L, c)
     for cell in range(L ** 4):
-        e = buf[hdr["cells_offset"] + cell * hdr["entry_bytes"]:][:2 * c]
-        assert list(np.frombuffer(e.tobytes(), dtype=np.uint16)) == list(ref[cell])
+        assert _cell_ids(buf, hdr, cell) == sorted(int(i) for i in ref[cell])
     assert abs(hdr["lo"] + R) < 1e-6 and abs(hdr["inv_h"] - L / (2 * R)) < 1e-3
 
 
