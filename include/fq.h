@@ -23,7 +23,8 @@
  *
  * Conventions for every entry point:
  *   - All array arguments are DEVICE pointers unless the comment says "host".  The caller owns
- *     every buffer; the library never allocates device memory and keeps no state between calls.
+ *     every buffer; the library never allocates device memory and keeps no state between calls
+ *     (fq_attn_decode_noalloc, below, is the one exception: it uses a fixed library array).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) and is
  *     asynchronous; results are valid once the stream has reached the enqueued work.
  *   - Errors are returned as fq_status from host-side validation before anything is enqueued,
@@ -130,6 +131,36 @@ fq_status fq_attn_decode(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, i
                          const float* rotV, const float* cbV,
                          float scale, float* out, void* workspace, size_t workspace_bytes,
                          void* stream);
+
+/* Size of the fixed device scratch used by fq_attn_decode_noalloc (4 MiB per GPU). */
+#define FQ_ATTN_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * fq_attn_decode_noalloc - fq_attn_decode for callers that cannot allocate device memory.
+ * (No counterpart in the paper: this is a convenience of this library.)
+ *
+ * fq_attn_decode needs a caller-owned workspace for its split-softmax partials.  Callers that
+ * cannot allocate one - code running inside a host application whose allocator owns all
+ * device memory, or a decode loop that must not call cudaMalloc because allocation may
+ * synchronise the device and has unbounded latency - can call this instead.  It keeps the
+ * partials in a fixed array of FQ_ATTN_NOALLOC_SCRATCH_BYTES that every GPU loading this
+ * library holds until the process exits, and it allocates nothing.
+ *   Arguments, layouts, limits and results are those of fq_attn_decode without the workspace.
+ *   Sizes whose fq_attn_workspace_bytes(...) exceeds FQ_ATTN_NOALLOC_SCRATCH_BYTES return
+ *   FQ_ERR_WORKSPACE before anything is enqueued.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress
+ *   with that device current); make that first call before any stream capture.
+ *   All calls on a device share the one array: calls that overlap on the GPU (for example on
+ *   two streams at once) race and give undefined results; calls ordered on one stream are
+ *   safe.  Nothing in the array needs to start at zero (every partial read is written first
+ *   by the same call).
+ */
+fq_status fq_attn_decode_noalloc(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int d,
+                                 const uint8_t* k_codes, const uint16_t* k_norms, int kK,
+                                 int NK, const float* rotK, const float* cbK,
+                                 const uint8_t* v_codes, const uint16_t* v_norms, int kV,
+                                 int NV, const float* rotV, const float* cbV, float scale,
+                                 float* out, void* stream);
 
 /*
  * fq_build_search_index - builds, on the HOST, the candidate table fq_encode can use instead

@@ -5,6 +5,7 @@ holds its thin ctypes binding (``_lib``), the table loader (``tables``), the see
 workloads (``workloads``) and the in-tree build step (``build``).  Importing the package does
 not load the library; the first compute call does, and raises if it is missing.
 """
-from ._lib import (FQ_F16, FQ_F32, FQ_INDEX_EXACT, FQ_INDEX_TOPC, FQError,  # noqa: F401
-                   fq_attn_decode, fq_attn_workspace_bytes, fq_build_search_index, fq_decode,
+from ._lib import (FQ_ATTN_NOALLOC_SCRATCH_BYTES, FQ_F16, FQ_F32, FQ_INDEX_EXACT,  # noqa: F401
+                   FQ_INDEX_TOPC, FQError,
+                   fq_attn_decode, fq_attn_decode_noalloc, fq_attn_workspace_bytes, fq_build_search_index, fq_decode,
                    fq_encode, fq_padded_dim, fq_payload_bytes, lib, status_string)

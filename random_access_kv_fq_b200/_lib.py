@@ -41,7 +41,13 @@ _SIGS = {
                             ctypes.c_float, _vp, _vp, _sz, _vp]),
     "fq_build_search_index": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _sz,
                                    ctypes.POINTER(_sz)]),
+    "fq_attn_decode_noalloc": (_i, [_vp, _i, _i, _i, _c_i64, _i,
+                                    _vp, _vp, _i, _i, _vp, _vp,
+                                    _vp, _vp, _i, _i, _vp, _vp,
+                                    ctypes.c_float, _vp, _vp]),
 }
+
+FQ_ATTN_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 _lib = None
 
@@ -168,6 +174,26 @@ def fq_attn_decode(q, k_codes, k_norms, kK: int, NK: int, rotK, cbK, v_codes, v_
                               float(scale), _ptr(out), _ptr(workspace), ws_bytes,
                               _stream(stream))
     _check("fq_attn_decode", st)
+    return out
+
+
+def fq_attn_decode_noalloc(q, k_codes, k_norms, kK: int, NK: int, rotK, cbK, v_codes, v_norms,
+                           kV: int, NV: int, rotV, cbV, scale: Optional[float] = None, out=None,
+                           stream=None):
+    """fq_attn_decode without a workspace argument: the library's fixed per-GPU scratch holds
+    the partials (for callers that cannot allocate device memory)."""
+    import torch
+    B, Hq, d = q.shape
+    _, Hkv, T, _ = k_codes.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    st = lib().fq_attn_decode_noalloc(_ptr(q), B, Hq, Hkv, T, d,
+                                      _ptr(k_codes), _ptr(k_norms), kK, NK, _ptr(rotK), _ptr(cbK),
+                                      _ptr(v_codes), _ptr(v_norms), kV, NV, _ptr(rotV), _ptr(cbV),
+                                      float(scale), _ptr(out), _stream(stream))
+    _check("fq_attn_decode_noalloc", st)
     return out
 
 
