@@ -257,7 +257,13 @@ size_t attn_smem_bytes(const AttnArgs& a) {
   return (size_t)smem_layout(a.Hq / a.Hkv, a.ks, a.vs).total * sizeof(float);
 }
 
+cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t st) {
+  attn_combine_kernel<<<dim3(a.Hq, a.B), 128, a.vs.dp * sizeof(float), st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+  if (attn100::supported(a)) return attn100::launch(a, st);
   size_t smem = attn_smem_bytes(a);
   cudaError_t e = cudaFuncSetAttribute(attn_partial_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -266,8 +272,7 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   attn_partial_kernel<<<grid, kThreads, smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<dim3(a.Hq, a.B), 128, a.vs.dp * sizeof(float), st>>>(a);
-  return cudaGetLastError();
+  return launch_attn_combine(a, st);
 }
 
 }  // namespace fq

@@ -82,34 +82,162 @@ __device__ __forceinline__ void group_sync(int g) {
   asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(128) : "memory");
 }
 
-// Nearest codeword of the normalised block zb among codewords ids (ascending); strict-less
-// keeps the lowest index on ties.
+// ---- nearest-codeword search policies ------------------------------------------------------
+// Scores are 1 + |c|^2 - 2 z.c: the squared distance minus |z|^2 (common to all candidates)
+// plus a constant.  Candidates are scanned in increasing index order with a strict less-than,
+// so equal distances keep the lowest index, as in the oracle.
+__device__ __forceinline__ void take_if_less(float s, int c, float& best, int& bi) {
+  const bool lt = s < best;
+  best = lt ? s : best;
+  bi = lt ? c : bi;
+}
+
+// score of codeword c from the shared-memory table (-2c, 1 + |c|^2)
 template <int K>
-__device__ __forceinline__ void consider(const float4* __restrict__ tbl, int c, const float (&zb)[K],
-                                         float& best, int& bi) {
-  float s;
+__device__ __forceinline__ float score_tbl(const float4* __restrict__ tbl, int c, const float (&zb)[K]) {
   if constexpr (K <= 3) {
-    float4 t = tbl[c];
-    s = t.w;
-    s = fmaf(zb[0], t.x, s);
+    const float4 t = tbl[c];
+    float s = fmaf(zb[0], t.x, t.w);
     if constexpr (K >= 2) s = fmaf(zb[1], t.y, s);
     if constexpr (K >= 3) s = fmaf(zb[2], t.z, s);
+    return s;
   } else {
-    float4 t = tbl[2 * c];
-    float4 u = tbl[2 * c + 1];
-    s = u.x;
-    s = fmaf(zb[0], t.x, s);
+    const float4 t = tbl[2 * c];
+    const float cc = tbl[2 * c + 1].x;
+    float s = fmaf(zb[0], t.x, cc);
     s = fmaf(zb[1], t.y, s);
     s = fmaf(zb[2], t.z, s);
-    s = fmaf(zb[3], t.w, s);
-  }
-  if (s < best) {
-    best = s;
-    bi = c;
+    return fmaf(zb[3], t.w, s);
   }
 }
 
-template <int K, int DP, int B>
+// flat grid cell: c_a = clamp(floor((z_a - lo) / h), 0, L - 1); the floor is a round-down add
+// of 2^23 (no conversion instruction)
+template <int K>
+__device__ __forceinline__ int grid_cell(const float (&zb)[K], float scale, float off, float top,
+                                         int L) {
+  int flat = 0, mul = 1;
+#pragma unroll
+  for (int a = 0; a < K; ++a) {
+    const float t = fminf(fmaxf(fmaf(zb[a], scale, off), 0.f), top);
+    flat += (__float_as_int(__fadd_rd(t, 8388608.0f)) - 0x4B000000) * mul;
+    mul *= L;
+  }
+  return flat;
+}
+
+struct GridParams {
+  const uint8_t* cells;
+  float scale, off, top;
+  int L, slots, entry, idb;
+};
+
+// Exact grid lists of at most 4W one-byte ids per cell in W 32-bit words (branch-free; the
+// padding repeats the last id, which cannot change the result).
+template <int K, int B, int W>
+struct SearchWords {
+  GridParams g;
+  const float4* tbl;
+  __device__ __forceinline__ int find(const float (&zb)[K]) const {
+    const uint32_t* e = reinterpret_cast<const uint32_t*>(g.cells) +
+                        (size_t)grid_cell<K>(zb, g.scale, g.off, g.top, g.L) * W;
+    uint32_t ids[W];
+    if constexpr (W == 2) {
+      const uint2 v = *reinterpret_cast<const uint2*>(e);
+      ids[0] = v.x;
+      ids[1] = v.y;
+    } else {
+#pragma unroll
+      for (int w = 0; w < W; ++w) ids[w] = e[w];
+    }
+    int bi = ids[0] & 0xFFu;
+    float best = score_tbl<K>(tbl, bi, zb);
+#pragma unroll
+    for (int q = 1; q < 4 * W; ++q) {
+      const int c = (ids[q / 4] >> (8 * (q % 4))) & 0xFFu;
+      take_if_less(score_tbl<K>(tbl, c, zb), c, best, bi);
+    }
+    return bi;
+  }
+};
+
+// Exact grid lists of any length (runtime slot count).
+template <int K, int B>
+struct SearchList {
+  GridParams g;
+  const float4* tbl;
+  __device__ __forceinline__ int find(const float (&zb)[K]) const {
+    const uint8_t* e =
+        g.cells + (size_t)grid_cell<K>(zb, g.scale, g.off, g.top, g.L) * g.entry;
+    float best = INFINITY;
+    int bi = 0;
+    for (int q = 0; q < g.slots; ++q) {
+      const int c = g.idb == 1 ? e[q] : reinterpret_cast<const uint16_t*>(e)[q];
+      take_if_less(score_tbl<K>(tbl, c, zb), c, best, bi);
+    }
+    return bi;
+  }
+};
+
+// All N codewords from the shared-memory table.
+template <int K, int B>
+struct SearchAll {
+  const float4* tbl;
+  int N;
+  __device__ __forceinline__ int find(const float (&zb)[K]) const {
+    float best = INFINITY;
+    int bi = 0;
+#pragma unroll 4
+    for (int c = 0; c < N; ++c) take_if_less(score_tbl<K>(tbl, c, zb), c, best, bi);
+    return bi;
+  }
+};
+
+// All N = 2^B <= 16 codewords held in registers; two candidates scored per packed FMA.
+template <int K, int B>
+struct SearchRegs {
+  static constexpr int N = 1 << B;
+  static constexpr int NP = (N + 1) / 2;
+  float2 m[NP][K];
+  float2 cc[NP];
+  __device__ __forceinline__ void load(const float4* __restrict__ tbl) {
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      float a[2][4], c2[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = (2 * q + h < N) ? 2 * q + h : 2 * q;
+        if constexpr (K <= 3) {
+          const float4 t = tbl[c];
+          a[h][0] = t.x; a[h][1] = t.y; a[h][2] = t.z; a[h][3] = 0.f;
+          c2[h] = t.w;
+        } else {
+          const float4 t = tbl[2 * c];
+          a[h][0] = t.x; a[h][1] = t.y; a[h][2] = t.z; a[h][3] = t.w;
+          c2[h] = tbl[2 * c + 1].x;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < K; ++k) m[q][k] = make_float2(a[0][k], a[1][k]);
+      cc[q] = make_float2(c2[0], c2[1]);
+    }
+  }
+  __device__ __forceinline__ int find(const float (&zb)[K]) const {
+    float best = INFINITY;
+    int bi = 0;
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      float2 s = cc[q];
+#pragma unroll
+      for (int k = 0; k < K; ++k) s = __ffma2_rn(make_float2(zb[k], zb[k]), m[q][k], s);
+      take_if_less(s.x, 2 * q, best, bi);
+      if (2 * q + 1 < N) take_if_less(s.y, 2 * q + 1, best, bi);
+    }
+    return bi;
+  }
+};
+
+template <int K, int DP, int B, bool GRID>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_f16_d64_kernel(const __grid_constant__ CUtensorMap xmap, EncParams p) {
   using C = EncCfg<K, DP, B>;
@@ -181,10 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<__half*>(sB + ptx::sw128_offset(2 * DP + (e >> 6), e & 63)) =
           __float2half_rn(0.f);
   }
-  // codebook table: (-2c, |c|^2) per codeword
+  // codebook table: (-2c, 1 + |c|^2) per codeword (see the search policies)
   for (int c = tid; c < p.N; c += kThreads) {
     float v[4] = {0.f, 0.f, 0.f, 0.f};
-    float cc = 0.f;
+    float cc = 1.f;
 #pragma unroll
     for (int a = 0; a < K; ++a) {
       v[a] = __ldg(p.cb + (size_t)c * K + a);
@@ -198,24 +326,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   // search index: used when it describes this (k, N, d') and has no overflow lists
-  bool use_ix = false;
-  const uint8_t* ix_cells = nullptr;
-  int ix_L = 0, ix_slots = 0, ix_entry = 0, ix_idb = 1;
-  bool ix_word = false;
-  float ix_scale = 0.f, ix_off = 0.f, ix_top = 0.f;
-  if (p.index != nullptr) {
+  int mode = 2;  // 0 / 3: four / eight one-byte ids per cell, 1: any list, 2: all codewords
+  GridParams gp{};
+  if (GRID && p.index != nullptr) {
     const IndexHeader h = *reinterpret_cast<const IndexHeader*>(p.index);
     if (h.magic == kIndexMagic && h.version == kIndexVersion && h.k == K && h.N == p.N &&
         h.dp == DP && !index_has_overflow(h)) {
-      use_ix = true;
-      ix_L = h.L;
-      ix_slots = h.slots;
-      ix_entry = h.entry_bytes;
-      ix_idb = h.id_bytes;
-      ix_scale = h.inv_h;
-      ix_off = -h.lo * h.inv_h;
-      ix_top = (float)(h.L - 1);
-      ix_word = h.id_bytes == 1 && h.entry_bytes == 4;
+      mode = (h.id_bytes == 1 && h.entry_bytes == 4) ? 0
+             : (h.id_bytes == 1 && h.entry_bytes == 8) ? 3 : 1;
+      gp.L = h.L;
+      gp.slots = h.slots;
+      gp.entry = h.entry_bytes;
+      gp.idb = h.id_bytes;
+      gp.scale = h.inv_h;
+      gp.off = -h.lo * h.inv_h;
+      gp.top = (float)(h.L - 1);
       const size_t bytes = (size_t)h.n_cells * h.entry_bytes;
       if (bytes <= (size_t)kIndexSmemBudget) {
         const uint4* src = reinterpret_cast<const uint4*>(p.index + h.cells_offset);
@@ -236,9 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (size_t i = (bytes / 16) * 16 + tid; i < bytes; i += kThreads)
           sIxSmem[i] = p.index[h.cells_offset + i];
-        ix_cells = sIxSmem;
+        gp.cells = sIxSmem;
       } else {
-        ix_cells = p.index + h.cells_offset;
+        gp.cells = p.index + h.cells_offset;
       }
     }
   }
@@ -271,6 +396,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  // The tile loop, instantiated once per search policy; the policy is chosen once per CTA so
+  // that only one version is hot in the instruction cache.
+  auto run = [&](const auto& search) {
   int i = 0;
   for (int64_t tile = first; tile < n_tiles; tile += stride, ++i) {
     const int s = i & 1;
@@ -345,32 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float zb[K];
 #pragma unroll
       for (int a = 0; a < K; ++a) zb[a] = z[j * K + a];
-      float best = INFINITY;
-      int bi = 0;
-      if (use_ix) {
-        // cell c_a = clamp(floor((z_a - lo) / h), 0, L - 1); the floor is the round-down add
-        // of 2^23 (no conversion instruction)
-        int flat = 0, mul = 1;
-#pragma unroll
-        for (int a = 0; a < K; ++a) {
-          const float t = fminf(fmaxf(fmaf(zb[a], ix_scale, ix_off), 0.f), ix_top);
-          flat += (__float_as_int(__fadd_rd(t, 8388608.0f)) - 0x4B000000) * mul;
-          mul *= ix_L;
-        }
-        const uint8_t* e = ix_cells + (size_t)flat * ix_entry;
-        if (ix_word) {  // four 1-byte ids in one 32-bit entry, branch-free (repeats are harmless)
-          const uint32_t ids = *reinterpret_cast<const uint32_t*>(e);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) consider<K>(sCb, (ids >> (8 * q)) & 0xFFu, zb, best, bi);
-        } else if (ix_idb == 1) {
-          for (int q = 0; q < ix_slots; ++q) consider<K>(sCb, e[q], zb, best, bi);
-        } else {
-          const uint16_t* e16 = reinterpret_cast<const uint16_t*>(e);
-          for (int q = 0; q < ix_slots; ++q) consider<K>(sCb, e16[q], zb, best, bi);
-        }
-      } else {
-        for (int c = 0; c < p.N; ++c) consider<K>(sCb, c, zb, best, bi);
-      }
+      const int bi = search.find(zb);
       const int off = j * B;  // compile-time after unrolling
       w[off / 32] |= (uint32_t)bi << (off % 32);
       if ((off % 32) + B > 32) w[off / 32 + 1] |= (uint32_t)bi >> (32 - off % 32);
@@ -408,6 +511,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(stage)[q];
     for (int q = (bytes / 16) * 16 + lt; q < bytes; q += 128) dst[q] = stage[q];
   }
+  };
+
+  if constexpr (!GRID && B <= 4) {
+    SearchRegs<K, B> sr;
+    sr.load(sCb);
+    run(sr);
+  } else {
+    if (mode == 0)
+      run(SearchWords<K, B, 1>{gp, sCb});
+    else if (mode == 3)
+      run(SearchWords<K, B, 2>{gp, sCb});
+    else if (mode == 1)
+      run(SearchList<K, B>{gp, sCb});
+    else
+      run(SearchAll<K, B>{sCb, p.N});
+  }
 
   ptx::tc_fence_before();
   __syncthreads();
@@ -437,6 +556,9 @@ struct DecParams {
   void* y;
 };
 
+constexpr int kDecGroups = 4;                // pipelines per decode CTA (16 warps per SM)
+constexpr int kDecThreads = 128 * kDecGroups;
+
 template <int K, int DP, int B, bool OUT_F16>
 struct DecCfg {
   static constexpr int M = DP / K;
@@ -450,10 +572,10 @@ struct DecCfg {
   // layout (1024-aligned offsets)
   static constexpr int OFF_B = 0;
   static constexpr int OFF_A = ((B_BYTES + 1023) / 1024) * 1024;
-  static constexpr int GROUP_BYTES = ((2 * A_BYTES + REC_BYTES + 1023) / 1024) * 1024;
-  static constexpr int OFF_CB = OFF_A + kGroups * GROUP_BYTES;
+  static constexpr int GROUP_BYTES = ((2 * A_BYTES + 2 * REC_BYTES + 1023) / 1024) * 1024;
+  static constexpr int OFF_CB = OFF_A + kDecGroups * GROUP_BYTES;
   static constexpr int OFF_BAR = OFF_CB + 256 * CBE;
-  static constexpr int SMEM = OFF_BAR + 128 + 1024;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
 };
 
 // fp16 hi part and 2^12-scaled fp16 lo part of v
@@ -463,46 +585,56 @@ __device__ __forceinline__ void split_f16(float v, __half& hi, __half& lo) {
 }
 
 template <int K, int DP, int B, bool OUT_F16>
-__global__ void __launch_bounds__(kThreads, 1) decode_d64_kernel(DecParams p) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_d64_kernel(DecParams p) {
   using C = DecCfg<K, DP, B, OUT_F16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = smem + C::OFF_B;
   uint8_t* sCb = smem + C::OFF_CB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 64);
-  int* sFlag = reinterpret_cast<int*>(smem + C::OFF_BAR + 72);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // per group: rec[2], mma
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 128);
+  int* sFlag = reinterpret_cast<int*>(smem + C::OFF_BAR + 144);
   const int tid = threadIdx.x, g = tid >> 7, lt = tid & 127, warp = tid >> 5;
   uint8_t* sAh = smem + C::OFF_A + g * C::GROUP_BYTES;
   uint8_t* sAl = sAh + C::A_BYTES;
-  uint8_t* sRec = sAl + C::A_BYTES;
+  uint8_t* sRec0 = sAl + C::A_BYTES;  // two record buffers of REC_BYTES
+  uint64_t* rec_full = bars + 3 * g;
+  const int64_t n_tiles = (p.n + kRows - 1) / kRows;
+  const int64_t stride = (int64_t)gridDim.x * kDecGroups;
+  const int64_t first = (int64_t)blockIdx.x * kDecGroups + g;
+  const int64_t n_full = p.n / kRows;  // tiles whose records are copied in bulk
+  auto issue_rec = [&](int64_t tile, int s) {
+    ptx::mbar_arrive_expect_tx(&rec_full[s], kRows * C::P);
+    ptx::bulk_load(sRec0 + s * C::REC_BYTES, p.codes + tile * kRows * C::P, kRows * C::P,
+                   &rec_full[s]);
+  };
 
   if (warp == 0) {
-    ptx::tmem_alloc(sTmem, 256);
+    ptx::tmem_alloc(sTmem, 512);
     ptx::tmem_relinquish();
   }
-  if (tid == 0) {
-    ptx::mbar_init(&bars[0], 1);
-    ptx::mbar_init(&bars[1], 1);
-    sFlag[0] = 0;
-    sFlag[1] = 0;
+  if (lt == 0) {  // each pipeline starts fetching its first records before the tables are built
+    for (int q = 0; q < 3; ++q) ptx::mbar_init(&bars[3 * g + q], 1);
+    sFlag[g] = 0;
     ptx::fence_mbar_init();
+    for (int s = 0; s < 2; ++s)
+      if (first + s * stride < n_full) issue_rec(first + s * stride, s);
   }
   // B operand rows c < 64: Pi^T_hi[c][r] = hi(Pi[r][c]); rows 64 + c: lo(Pi[r][c]); r < d'.
   // Pi is read row-major (coalesced, all loads issued first) and written transposed.
   {
     constexpr int kElems = DP * 64;
-    constexpr int kIter = (kElems + kThreads - 1) / kThreads;
+    constexpr int kIter = (kElems + kDecThreads - 1) / kDecThreads;
     float v[kIter];
 #pragma unroll
     for (int it = 0; it < kIter; ++it) {
-      const int e = tid + it * kThreads;
+      const int e = tid + it * kDecThreads;
       if (e < kElems) v[it] = __ldg(p.rot + (size_t)(e >> 6) * DP + (e & 63));
     }
 #pragma unroll
     for (int it = 0; it < kIter; ++it) {
-      const int e = tid + it * kThreads;
+      const int e = tid + it * kDecThreads;
       if (e < kElems) {
         const int r = e >> 6, c = e & 63;
         __half hi, lo;
@@ -517,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_d64_kernel(DecParams p) {
       }
     }
     if constexpr (C::EXTRA) {  // K columns d'..79 of the fifth step are zero
-      for (int e = tid; e < 128 * (C::KSTEPS * 16 - DP); e += kThreads) {
+      for (int e = tid; e < 128 * (C::KSTEPS * 16 - DP); e += kDecThreads) {
         const int row = e / (C::KSTEPS * 16 - DP), r = DP + e % (C::KSTEPS * 16 - DP);
         *reinterpret_cast<__half*>(sB + 128 * 128 + ptx::noswz16_offset(row, r - 64)) =
             __float2half_rn(0.f);
@@ -525,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_d64_kernel(DecParams p) {
     }
   }
   // codeword table: fp16 hi / lo parts of each coordinate
-  for (int c = tid; c < p.N; c += kThreads) {
+  for (int c = tid; c < p.N; c += kDecThreads) {
     __half hi[4], lo[4];
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
@@ -558,25 +690,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_d64_kernel(DecParams p) {
   ptx::tc_fence_after();
   const uint32_t tmem = *sTmem;
   const uint32_t acc = tmem + g * 128;
-  uint64_t* mma_bar = &bars[g];
+  uint64_t* mma_bar = &bars[3 * g + 2];
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   constexpr uint32_t idesc128 = ptx::idesc_f16_f32(128, 128);
   constexpr uint32_t idesc64 = ptx::idesc_f16_f32(128, 64);
   const uint32_t aH = ptx::smem_u32(sAh), aL = ptx::smem_u32(sAl), bA = ptx::smem_u32(sB);
 
-  const int64_t n_tiles = (p.n + kRows - 1) / kRows;
-  const int64_t stride = (int64_t)gridDim.x * kGroups;
   int i = 0;
-  for (int64_t tile = (int64_t)blockIdx.x * kGroups + g; tile < n_tiles; tile += stride, ++i) {
+  for (int64_t tile = first; tile < n_tiles; tile += stride, ++i) {
     const int64_t rem = p.n - tile * kRows;
     const int rows = rem < kRows ? (int)rem : kRows;
-    // stage the tile's records
-    const uint8_t* src = p.codes + tile * kRows * C::P;
-    const int bytes = rows * C::P;
-    for (int q = lt; q < bytes / 16; q += 128)
-      reinterpret_cast<uint4*>(sRec)[q] = __ldg(reinterpret_cast<const uint4*>(src) + q);
-    for (int q = (bytes / 16) * 16 + lt; q < bytes; q += 128) sRec[q] = src[q];
-    group_sync(g);
+    const int s = i & 1;
+    uint8_t* sRec = sRec0 + s * C::REC_BYTES;
+    const float nu = (lt < rows) ? f16_bits_to_f32(p.norms[tile * kRows + lt]) : 0.f;
+    if (tile < n_full) {  // records arrive by bulk copy
+      if (!ptx::mbar_wait(&rec_full[s], (i >> 1) & 1)) sFlag[g] = 1;
+    } else {  // the ragged last tile: plain loads
+      const uint8_t* src = p.codes + tile * kRows * C::P;
+      const int bytes = rows * C::P;
+      for (int q = lt; q < bytes / 16; q += 128)
+        reinterpret_cast<uint4*>(sRec)[q] = __ldg(reinterpret_cast<const uint4*>(src) + q);
+      for (int q = (bytes / 16) * 16 + lt; q < bytes; q += 128) sRec[q] = src[q];
+      group_sync(g);
+    }
     // unpack, gather, split into the A tiles
     uint32_t w[(C::P + 3) / 4 + 1];
 #pragma unroll
@@ -595,58 +731,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_d64_kernel(DecParams p) {
         for (int q = 0; q < C::P; ++q) w[q / 4] |= uint32_t(rec[q]) << (8 * (q & 3));
       }
     }
-    uint32_t hw[(DP + 1) / 2 + 1], lw[(DP + 1) / 2 + 1];  // half2 words of zhat hi / lo
+    // gather codewords and write the A tiles one 16-byte chunk (8 coordinates) at a time
+    constexpr int NCH = (DP + 7) / 8;
 #pragma unroll
-    for (int q = 0; q < (DP + 1) / 2 + 1; ++q) hw[q] = lw[q] = 0u;
+    for (int c = 0; c < NCH; ++c) {
+      uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
+      const int j0 = (8 * c) / K;
+      const int j1 = ((8 * c + 7) / K < C::M - 1) ? (8 * c + 7) / K : C::M - 1;
 #pragma unroll
-    for (int j = 0; j < C::M; ++j) {
-      const int off = j * B;
-      uint32_t id = w[off / 32] >> (off % 32);
-      if ((off % 32) + B > 32) id |= w[off / 32 + 1] << (32 - off % 32);
-      id &= (1u << B) - 1u;
-      if constexpr (K == 2) {
-        const uint2 e = *reinterpret_cast<const uint2*>(sCb + id * 8);
-        hw[j] = e.x;
-        lw[j] = e.y;
-      } else {
-        const uint4 e = *reinterpret_cast<const uint4*>(sCb + id * 16);
-        const uint32_t h01 = e.x, h23 = e.y, l01 = e.z, l23 = e.w;
-        if constexpr (K == 4) {
-          hw[2 * j] = h01;
-          hw[2 * j + 1] = h23;
-          lw[2 * j] = l01;
-          lw[2 * j + 1] = l23;
-        } else {  // K == 3: halves 3j, 3j+1, 3j+2
-          const int h0 = 3 * j;
-          const uint32_t hv[3] = {h01 & 0xFFFFu, h01 >> 16, h23 & 0xFFFFu};
-          const uint32_t lv[3] = {l01 & 0xFFFFu, l01 >> 16, l23 & 0xFFFFu};
+      for (int j = j0; j <= j1; ++j) {
+        const int off = j * B;
+        uint32_t id = w[off / 32] >> (off % 32);
+        if ((off % 32) + B > 32) id |= w[off / 32 + 1] << (32 - off % 32);
+        id &= (1u << B) - 1u;
+        uint32_t eh[2], el[2];  // hi / lo half2 words of the codeword (up to 4 halves each)
+        if constexpr (K == 2) {
+          const uint2 e = *reinterpret_cast<const uint2*>(sCb + id * 8);
+          eh[0] = e.x; eh[1] = 0u; el[0] = e.y; el[1] = 0u;
+        } else {
+          const uint4 e = *reinterpret_cast<const uint4*>(sCb + id * 16);
+          eh[0] = e.x; eh[1] = e.y; el[0] = e.z; el[1] = e.w;
+        }
 #pragma unroll
-          for (int a = 0; a < 3; ++a) {
-            const int hh = h0 + a;
-            hw[hh / 2] |= hv[a] << (16 * (hh & 1));
-            lw[hh / 2] |= lv[a] << (16 * (hh & 1));
+        for (int a = 0; a < K; ++a) {
+          const int hp = K * j + a;
+          if (hp >= 8 * c && hp < 8 * c + 8) {
+            const int q = hp - 8 * c;
+            const uint32_t hh = (eh[a >> 1] >> (16 * (a & 1))) & 0xFFFFu;
+            const uint32_t ll = (el[a >> 1] >> (16 * (a & 1))) & 0xFFFFu;
+            hw[q >> 1] |= hh << (16 * (q & 1));
+            lw[q >> 1] |= ll << (16 * (q & 1));
           }
         }
       }
+      if (c < 8) {
+        *reinterpret_cast<uint4*>(sAh + ptx::sw128_offset(lt, 8 * c)) =
+            make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(sAl + ptx::sw128_offset(lt, 8 * c)) =
+            make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      } else {
+        *reinterpret_cast<uint4*>(sAh + kRows * 128 + ptx::noswz16_offset(lt, 0)) =
+            make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(sAl + kRows * 128 + ptx::noswz16_offset(lt, 0)) =
+            make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
     }
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      *reinterpret_cast<uint4*>(sAh + ptx::sw128_offset(lt, 8 * c)) =
-          make_uint4(hw[4 * c], hw[4 * c + 1], hw[4 * c + 2], hw[4 * c + 3]);
-      *reinterpret_cast<uint4*>(sAl + ptx::sw128_offset(lt, 8 * c)) =
-          make_uint4(lw[4 * c], lw[4 * c + 1], lw[4 * c + 2], lw[4 * c + 3]);
-    }
-    if constexpr (C::EXTRA) {
-      *reinterpret_cast<uint4*>(sAh + kRows * 128 + ptx::noswz16_offset(lt, 0)) =
-          make_uint4(hw[32], 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(sAl + kRows * 128 + ptx::noswz16_offset(lt, 0)) =
-          make_uint4(lw[32], 0u, 0u, 0u);
-    }
-    const float nu = (lt < rows) ? f16_bits_to_f32(p.norms[tile * kRows + lt]) : 0.f;
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
-    group_sync(g);
+    group_sync(g);  // A tiles written; this tile's records no longer read
     if (lt == 0) {
+      if (tile + 2 * stride < n_full) issue_rec(tile + 2 * stride, s);
       ptx::tc_fence_after();
 #pragma unroll
       for (int ks = 0; ks < C::KSTEPS; ++ks) {
@@ -713,8 +847,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_d64_kernel(DecParams p) {
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (tid == 0 && (sFlag[0] | sFlag[1])) atomicAdd(&g_fq_wait_timeouts, 1u);
-  if (warp == 0) ptx::tmem_dealloc(tmem, 256);
+  if (tid == 0 && (sFlag[0] | sFlag[1] | sFlag[2] | sFlag[3]))
+    atomicAdd(&g_fq_wait_timeouts, 1u);
+  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
 }
 
 // ---- host side --------------------------------------------------------------------------------
@@ -747,8 +882,8 @@ bool is_sm100() {
   return major == 10;
 }
 
-template <int K, int DP, int B>
-cudaError_t launch_enc(const void* x, int64_t n, const EncParams& p, cudaStream_t st) {
+template <int K, int DP, int B, bool GRID>
+cudaError_t launch_enc_kernel(const void* x, int64_t n, const EncParams& p, cudaStream_t st) {
   using C = EncCfg<K, DP, B>;
   CUtensorMap map;
   const cuuint64_t dims[2] = {64, (cuuint64_t)n};
@@ -761,13 +896,19 @@ cudaError_t launch_enc(const void* x, int64_t n, const EncParams& p, cudaStream_
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = encode_f16_d64_kernel<K, DP, B>;
+  auto kern = encode_f16_d64_kernel<K, DP, B, GRID>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (n + kRows - 1) / kRows;
   const int64_t ctas = std::min<int64_t>((tiles + kGroups - 1) / kGroups, sm_count());
   kern<<<(int)ctas, kThreads, C::SMEM, st>>>(map, p);
   return cudaGetLastError();
+}
+
+template <int K, int DP, int B>
+cudaError_t launch_enc(const void* x, int64_t n, const EncParams& p, cudaStream_t st) {
+  if (p.index != nullptr) return launch_enc_kernel<K, DP, B, true>(x, n, p, st);
+  return launch_enc_kernel<K, DP, B, false>(x, n, p, st);
 }
 
 template <int K, int DP, int B, bool F16>
@@ -777,8 +918,8 @@ cudaError_t launch_dec(const DecParams& p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (p.n + kRows - 1) / kRows;
-  const int64_t ctas = std::min<int64_t>((tiles + kGroups - 1) / kGroups, sm_count());
-  kern<<<(int)ctas, kThreads, C::SMEM, st>>>(p);
+  const int64_t ctas = std::min<int64_t>((tiles + kDecGroups - 1) / kDecGroups, sm_count());
+  kern<<<(int)ctas, kDecThreads, C::SMEM, st>>>(p);
   return cudaGetLastError();
 }
 

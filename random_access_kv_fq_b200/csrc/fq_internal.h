@@ -102,5 +102,12 @@ int64_t attn_tokens_per_split(int64_t T, int splits);
 size_t attn_partials_bytes(int B, int Hq, int splits, int dpV);
 size_t attn_smem_bytes(const AttnArgs& a);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t st);
+
+// sm_100a tensor-core attention (attn_sm100.cu) for the shapes it supports.
+namespace attn100 {
+bool supported(const AttnArgs& a);
+cudaError_t launch(const AttnArgs& a, cudaStream_t st);
+}  // namespace attn100
 
 }  // namespace fq

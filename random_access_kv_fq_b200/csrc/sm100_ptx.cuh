@@ -10,9 +10,9 @@
 namespace fq {
 namespace ptx {
 
-// A wait gives up after this many polls (~64 ns apart): a bug or a hung copy turns into
-// an error flag instead of a hung GPU.
-constexpr uint32_t kSpinLimit = 1u << 24;
+// A wait gives up after this many try_wait attempts (each suspends the thread for at most a
+// hardware time limit): a bug or a hung copy turns into an error flag instead of a hung GPU.
+constexpr uint32_t kSpinLimit = 1u << 20;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -45,12 +45,22 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete; false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
-    if (mbar_test(bar, parity)) return true;
-    if (it >= 16) __nanosleep(64);
-  }
+  for (uint32_t it = 0; it < kSpinLimit; ++it)
+    if (mbar_try(bar, parity)) return true;
   return false;
 }
 
@@ -61,6 +71,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Untiled bulk copy global -> shared (both addresses 16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes),
+      "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -120,6 +140,20 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
          | (uint32_t(M >> 4) << 24);         // M / 16
 }
 
+// Same with the A operand stored MN-major (M contiguous), B K-major.
+__host__ __device__ constexpr uint32_t idesc_f16_f32_amn(int M, int N) {
+  return idesc_f16_f32(M, N) | (1u << 15);
+}
+
+// Descriptor of an MN-major operand stored with the 128-byte swizzle: 64 contiguous M
+// elements (128 B) per K row, 8 K rows per 1024-byte atom, `lbo` bytes between M atoms and
+// `sbo` bytes between groups of 8 K rows.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t addr, uint32_t lbo,
+                                                        uint32_t sbo) {
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
 // Shared-memory matrix descriptor of a K-major operand stored with the 128-byte swizzle
 // (8-row groups of 128-byte rows, groups 1024 bytes apart).  `addr` is the shared address
 // of the first element the MMA reads (the group base must be 1024-byte aligned; K offsets
@@ -168,6 +202,19 @@ __device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t (&r)[2]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
                : "=r"(r[0]), "=r"(r[1])
                : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32"
+      " [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");

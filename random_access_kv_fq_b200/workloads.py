@@ -106,7 +106,7 @@ GPT2 = CodecWorkload(
     "gpt2small_12Lx12Hx1024T_d64",
     CacheShape(batch=1, layers=12, heads=12, tokens=1024, d=64, sigma=1.0, outliers=True,
                dtype="f16", seed=1002),
-    (Rate(3, 64, "exact", grid_L=16, grid_c=10), Rate(4, 8, "brute")),
+    (Rate(3, 64, "exact", grid_L=20, grid_c=8), Rate(4, 8, "brute")),
 )
 TINYLLAMA = CodecWorkload(
     "tinyllama_22Lx4Hx2048Tx8B_d64",

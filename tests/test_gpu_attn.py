@@ -131,3 +131,35 @@ def test_attention_full_size_sampled():
                              rv, cv, 3, 64)
         ref = fo.attention_decoded(q[b:b + 1, g * G:(g + 1) * G], Kc, Vc, w.d, 1 / math.sqrt(w.d))
         par.check_attention(out[b:b + 1, g * G:(g + 1) * G], ref)
+
+
+@pytest.mark.parametrize("hq,hkv,T", [(16, 2, 1), (16, 2, 129), (16, 2, 1000), (32, 2, 700),
+                                      (8, 1, 5000), (16, 1, 256)])
+def test_attention_tensor_core_groups(hq, hkv, T):
+    """Group sizes 8 and 16 take the tensor-core kernel: ragged tiles, one token, long splits."""
+    w = wl.small_attn(batch=2, hq=hq, hkv=hkv, tokens=T, seed=hq + T)
+    q, Kc, Vc, _, _ = _setup(w)
+    for scale in (1 / math.sqrt(w.d), 0.5):
+        ref = fo.attention_decoded(q, Kc, Vc, w.d, scale)
+        par.check_attention(_gpu_attn(q, Kc, Vc, scale), ref)
+
+
+def test_attention_tensor_core_degenerate():
+    """T = 1 returns the decoded value; q = 0 returns the mean of the decoded values (G = 8)."""
+    w = wl.small_attn(batch=2, hq=16, hkv=2, tokens=1, seed=12)
+    q, Kc, Vc, _, _ = _setup(w)
+    vdec = fo.decode(Vc.codes.reshape(-1, Vc.codes.shape[-1]), Vc.norms.reshape(-1), Vc.rot,
+                     Vc.codebook, w.d, Vc.k, Vc.N).reshape(w.batch, w.hkv, 1, w.d)
+    out = _gpu_attn(q, Kc, Vc, 0.125)
+    for b in range(w.batch):
+        for h in range(w.hq):
+            np.testing.assert_allclose(out[b, h], vdec[b, h // 8, 0], rtol=1e-5,
+                                       atol=1e-5 * np.abs(vdec).max())
+    w2 = wl.small_attn(batch=2, hq=16, hkv=2, tokens=777, seed=13)
+    q2, Kc2, Vc2, _, _ = _setup(w2)
+    out2 = _gpu_attn(np.zeros_like(q2), Kc2, Vc2, 0.125)
+    vdec2 = fo.decode(Vc2.codes.reshape(-1, Vc2.codes.shape[-1]), Vc2.norms.reshape(-1), Vc2.rot,
+                      Vc2.codebook, w2.d, Vc2.k, Vc2.N).reshape(w2.batch, w2.hkv, 777, w2.d)
+    mean = vdec2.mean(axis=2)
+    for h in range(w2.hq):
+        par.check_attention(out2[:, h:h + 1], mean[:, h // 8][:, None])
