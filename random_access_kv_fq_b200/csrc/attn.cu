@@ -24,7 +24,10 @@ constexpr int kThreads = 256;
 constexpr int kTile = 64;       // tokens per tile
 constexpr int kAccPer = 9;      // accumulator entries per thread: 16 heads * 135 / 256
 constexpr int kMaxGroup = 16;
-constexpr int kTargetCtas = 148 * 4;
+// Context splits: one wave of the tensor-core kernel (three 128-token-tile CTAs per SM on the
+// 148 SMs of a B200), split lengths a multiple of 128 tokens.
+constexpr int kTargetCtas = 148 * 3;
+constexpr int kSplitGrain = 128;
 
 struct SmemLayout {
   int qt, lut, cv, S, kid, vid, kn, vn, alpha, mrun, lrun, total;  // float offsets
@@ -235,8 +238,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AttnArgs a) {
 
 int attn_splits(int B, int Hkv, int64_t T) {
   int64_t pairs = (int64_t)B * Hkv;
-  int64_t want = (kTargetCtas + pairs - 1) / pairs;
-  int64_t tiles = (T + kTile - 1) / kTile;
+  int64_t want = kTargetCtas / pairs;
+  int64_t tiles = (T + kSplitGrain - 1) / kSplitGrain;
   if (want > tiles) want = tiles;
   if (want < 1) want = 1;
   if (want > 4096) want = 4096;
@@ -246,7 +249,7 @@ int attn_splits(int B, int Hkv, int64_t T) {
 
 int64_t attn_tokens_per_split(int64_t T, int splits) {
   int64_t tps = (T + splits - 1) / splits;
-  return ((tps + kTile - 1) / kTile) * kTile;
+  return ((tps + kSplitGrain - 1) / kSplitGrain) * kSplitGrain;
 }
 
 size_t attn_partials_bytes(int B, int Hq, int splits, int dpV) {

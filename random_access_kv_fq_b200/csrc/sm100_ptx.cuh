@@ -124,6 +124,19 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 inputs, fp32 accumulate; one thread issues.  A is
+// M = 128 lanes (row i in lane i) with two fp16 K elements per 32-bit column, the even K
+// element in the low half; a_tmem addresses the column of the first K element.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when all previously issued UMMAs of this thread have completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -198,6 +211,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t (&r)[1]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t (&r)[2]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
                : "=r"(r[0]), "=r"(r[1])
@@ -216,6 +243,41 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+// Loads COUNT consecutive 32-bit columns starting at column offset START (both compile-time)
+// of this warp's 32 lanes into out[0..COUNT).
+template <int START, int COUNT>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* out) {
+  if constexpr (COUNT >= 16) {
+    uint32_t r[16];
+    tmem_ld16(taddr + START, r);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) out[i] = r[i];
+    tmem_ld_cols<START + 16, COUNT - 16>(taddr, out + 16);
+  } else if constexpr (COUNT >= 8) {
+    uint32_t r[8];
+    tmem_ld8(taddr + START, r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = r[i];
+    tmem_ld_cols<START + 8, COUNT - 8>(taddr, out + 8);
+  } else if constexpr (COUNT >= 4) {
+    uint32_t r[4];
+    tmem_ld4(taddr + START, r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) out[i] = r[i];
+    tmem_ld_cols<START + 4, COUNT - 4>(taddr, out + 4);
+  } else if constexpr (COUNT >= 2) {
+    uint32_t r[2];
+    tmem_ld2(taddr + START, r);
+    out[0] = r[0];
+    out[1] = r[1];
+    tmem_ld_cols<START + 2, COUNT - 2>(taddr, out + 2);
+  } else if constexpr (COUNT == 1) {
+    uint32_t r[1];
+    tmem_ld1(taddr + START, r);
+    out[0] = r[0];
+  }
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }

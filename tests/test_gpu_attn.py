@@ -163,3 +163,31 @@ def test_attention_tensor_core_degenerate():
     mean = vdec2.mean(axis=2)
     for h in range(w2.hq):
         par.check_attention(out2[:, h:h + 1], mean[:, h // 8][:, None])
+
+
+def _misaligned(a, shift_elems):
+    """A device copy of `a` whose data pointer sits `shift_elems` elements past an aligned
+    allocation (odd byte offsets for records, 2-byte offsets for norms)."""
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    buf = torch.empty(t.numel() + shift_elems, dtype=t.dtype, device="cuda")
+    view = buf[shift_elems:].view(t.shape)
+    view.copy_(t.cuda())
+    return view
+
+
+@pytest.mark.parametrize("hq,hkv,T,shift", [(16, 2, 1040, 1), (16, 2, 333, 3), (32, 2, 4112, 5),
+                                            (8, 1, 700, 7)])
+def test_attention_misaligned_caches(hq, hkv, T, shift):
+    """Records and norms at arbitrary (byte / element) offsets: tiles whose aligned bulk-copy
+    window would leave the buffer are read from global memory directly."""
+    w = wl.small_attn(batch=2, hq=hq, hkv=hkv, tokens=T, seed=3 * T + shift)
+    q, Kc, Vc, _, _ = _setup(w)
+    scale = 1 / math.sqrt(w.d)
+    out = fq.fq_attn_decode(_dev(q), _misaligned(Kc.codes, shift),
+                            _misaligned(Kc.norms.view(np.int16), 1), Kc.k, Kc.N, _dev(Kc.rot),
+                            _dev(Kc.codebook), _misaligned(Vc.codes, shift + 2),
+                            _misaligned(Vc.norms.view(np.int16), 3), Vc.k, Vc.N, _dev(Vc.rot),
+                            _dev(Vc.codebook), scale=scale)
+    torch.cuda.synchronize()
+    ref = fo.attention_decoded(q, Kc, Vc, w.d, scale)
+    par.check_attention(par.to_np(out), ref)
