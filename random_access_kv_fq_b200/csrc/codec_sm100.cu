@@ -534,324 +534,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
-// ================================================================================================
-// Decode (summary sec. 2.3, decoder): y = nu (Pi^T zhat)[0:64] for fp16 or fp32 output.
-//   records  the tile's 128 records staged in shared memory with 16-byte loads
-//   gather   each thread unpacks its indices and writes its row of zhat, split into fp16
-//            hi and lo parts (zhat = hi + 2^-12 lo), into the two UMMA A tiles
-//   tcgen05  D[:, 0:128]  = Zhi * [PiT_hi ; PiT_lo]^T     (one chain, N = 128)
-//            D[:, 64:128] += Zlo * PiT_hi^T               (second chain, N = 64)
-//            so that y = nu (D[:, 0:64] + 2^-12 D[:, 64:128]) carries ~22 bits
-//   store    each thread converts its row and writes it with 16-byte stores
-// d' = 66 (k = 3) adds a fifth K step whose operands use the no-swizzle layout.
-// ================================================================================================
-
-struct DecParams {
-  int64_t n;
-  int N;
-  const float* rot;
-  const float* cb;
-  const uint8_t* codes;
-  const uint16_t* norms;
-  void* y;
-};
-
-constexpr int kDecGroups = 4;                // pipelines per decode CTA (16 warps per SM)
-constexpr int kDecThreads = 128 * kDecGroups;
-
-template <int K, int DP, int B, bool OUT_F16>
-struct DecCfg {
-  static constexpr int M = DP / K;
-  static constexpr int P = (M * B + 7) / 8;
-  static constexpr int KSTEPS = (DP + 15) / 16;          // 4 (d' = 64) or 5 (d' = 66)
-  static constexpr bool EXTRA = KSTEPS > 4;             // fifth step in the no-swizzle layout
-  static constexpr int A_BYTES = kRows * 128 + (EXTRA ? kRows * 32 : 0);
-  static constexpr int B_BYTES = 128 * 128 + (EXTRA ? 128 * 32 : 0);
-  static constexpr int REC_BYTES = ((kRows * P + 15) / 16) * 16;
-  static constexpr int CBE = (K == 2) ? 8 : 16;         // bytes per codeword table entry
-  // layout (1024-aligned offsets)
-  static constexpr int OFF_B = 0;
-  static constexpr int OFF_A = ((B_BYTES + 1023) / 1024) * 1024;
-  static constexpr int GROUP_BYTES = ((2 * A_BYTES + 2 * REC_BYTES + 1023) / 1024) * 1024;
-  static constexpr int OFF_CB = OFF_A + kDecGroups * GROUP_BYTES;
-  static constexpr int OFF_BAR = OFF_CB + 256 * CBE;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
-};
-
-// fp16 hi part and 2^12-scaled fp16 lo part of v
-__device__ __forceinline__ void split_f16(float v, __half& hi, __half& lo) {
-  hi = __float2half_rn(v);
-  lo = __float2half_rn((v - __half2float(hi)) * 4096.0f);
-}
-
-template <int K, int DP, int B, bool OUT_F16>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_d64_kernel(DecParams p) {
-  using C = DecCfg<K, DP, B, OUT_F16>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sB = smem + C::OFF_B;
-  uint8_t* sCb = smem + C::OFF_CB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // per group: rec[2], mma
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 128);
-  int* sFlag = reinterpret_cast<int*>(smem + C::OFF_BAR + 144);
-  const int tid = threadIdx.x, g = tid >> 7, lt = tid & 127, warp = tid >> 5;
-  uint8_t* sAh = smem + C::OFF_A + g * C::GROUP_BYTES;
-  uint8_t* sAl = sAh + C::A_BYTES;
-  uint8_t* sRec0 = sAl + C::A_BYTES;  // two record buffers of REC_BYTES
-  uint64_t* rec_full = bars + 3 * g;
-  const int64_t n_tiles = (p.n + kRows - 1) / kRows;
-  const int64_t stride = (int64_t)gridDim.x * kDecGroups;
-  const int64_t first = (int64_t)blockIdx.x * kDecGroups + g;
-  const int64_t n_full = p.n / kRows;  // tiles whose records are copied in bulk
-  auto issue_rec = [&](int64_t tile, int s) {
-    ptx::mbar_arrive_expect_tx(&rec_full[s], kRows * C::P);
-    ptx::bulk_load(sRec0 + s * C::REC_BYTES, p.codes + tile * kRows * C::P, kRows * C::P,
-                   &rec_full[s]);
-  };
-
-  if (warp == 0) {
-    ptx::tmem_alloc(sTmem, 512);
-    ptx::tmem_relinquish();
-  }
-  if (lt == 0) {  // each pipeline starts fetching its first records before the tables are built
-    for (int q = 0; q < 3; ++q) ptx::mbar_init(&bars[3 * g + q], 1);
-    sFlag[g] = 0;
-    ptx::fence_mbar_init();
-    for (int s = 0; s < 2; ++s)
-      if (first + s * stride < n_full) issue_rec(first + s * stride, s);
-  }
-  // B operand rows c < 64: Pi^T_hi[c][r] = hi(Pi[r][c]); rows 64 + c: lo(Pi[r][c]); r < d'.
-  // Pi is read row-major (coalesced, all loads issued first) and written transposed.
-  {
-    constexpr int kElems = DP * 64;
-    constexpr int kIter = (kElems + kDecThreads - 1) / kDecThreads;
-    float v[kIter];
-#pragma unroll
-    for (int it = 0; it < kIter; ++it) {
-      const int e = tid + it * kDecThreads;
-      if (e < kElems) v[it] = __ldg(p.rot + (size_t)(e >> 6) * DP + (e & 63));
-    }
-#pragma unroll
-    for (int it = 0; it < kIter; ++it) {
-      const int e = tid + it * kDecThreads;
-      if (e < kElems) {
-        const int r = e >> 6, c = e & 63;
-        __half hi, lo;
-        split_f16(v[it], hi, lo);
-        if (r < 64) {
-          *reinterpret_cast<__half*>(sB + ptx::sw128_offset(c, r)) = hi;
-          *reinterpret_cast<__half*>(sB + ptx::sw128_offset(64 + c, r)) = lo;
-        } else {
-          *reinterpret_cast<__half*>(sB + 128 * 128 + ptx::noswz16_offset(c, r - 64)) = hi;
-          *reinterpret_cast<__half*>(sB + 128 * 128 + ptx::noswz16_offset(64 + c, r - 64)) = lo;
-        }
-      }
-    }
-    if constexpr (C::EXTRA) {  // K columns d'..79 of the fifth step are zero
-      for (int e = tid; e < 128 * (C::KSTEPS * 16 - DP); e += kDecThreads) {
-        const int row = e / (C::KSTEPS * 16 - DP), r = DP + e % (C::KSTEPS * 16 - DP);
-        *reinterpret_cast<__half*>(sB + 128 * 128 + ptx::noswz16_offset(row, r - 64)) =
-            __float2half_rn(0.f);
-      }
-    }
-  }
-  // codeword table: fp16 hi / lo parts of each coordinate
-  for (int c = tid; c < p.N; c += kDecThreads) {
-    __half hi[4], lo[4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      hi[a] = __float2half_rn(0.f);
-      lo[a] = hi[a];
-      if (a < K) split_f16(__ldg(p.cb + (size_t)c * K + a), hi[a], lo[a]);
-    }
-    if constexpr (K == 2) {
-      __half2* e = reinterpret_cast<__half2*>(sCb + c * 8);
-      e[0] = __halves2half2(hi[0], hi[1]);
-      e[1] = __halves2half2(lo[0], lo[1]);
-    } else {
-      __half2* e = reinterpret_cast<__half2*>(sCb + c * 16);
-      e[0] = __halves2half2(hi[0], hi[1]);
-      e[1] = __halves2half2(hi[2], hi[3]);
-      e[2] = __halves2half2(lo[0], lo[1]);
-      e[3] = __halves2half2(lo[2], lo[3]);
-    }
-  }
-  if constexpr (C::EXTRA) {  // zero the second 8-column core matrix of the fifth K step once
-    for (int row = lt; row < kRows; row += 128) {
-      *reinterpret_cast<uint4*>(sAh + kRows * 128 + ptx::noswz16_offset(row, 8)) = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(sAl + kRows * 128 + ptx::noswz16_offset(row, 8)) = make_uint4(0, 0, 0, 0);
-    }
-  }
-
-  ptx::fence_proxy_async_smem();
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-  const uint32_t tmem = *sTmem;
-  const uint32_t acc = tmem + g * 128;
-  uint64_t* mma_bar = &bars[3 * g + 2];
-  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  constexpr uint32_t idesc128 = ptx::idesc_f16_f32(128, 128);
-  constexpr uint32_t idesc64 = ptx::idesc_f16_f32(128, 64);
-  const uint32_t aH = ptx::smem_u32(sAh), aL = ptx::smem_u32(sAl), bA = ptx::smem_u32(sB);
-
-  int i = 0;
-  for (int64_t tile = first; tile < n_tiles; tile += stride, ++i) {
-    const int64_t rem = p.n - tile * kRows;
-    const int rows = rem < kRows ? (int)rem : kRows;
-    const int s = i & 1;
-    uint8_t* sRec = sRec0 + s * C::REC_BYTES;
-    const float nu = (lt < rows) ? f16_bits_to_f32(p.norms[tile * kRows + lt]) : 0.f;
-    if (tile < n_full) {  // records arrive by bulk copy
-      if (!ptx::mbar_wait(&rec_full[s], (i >> 1) & 1)) sFlag[g] = 1;
-    } else {  // the ragged last tile: plain loads
-      const uint8_t* src = p.codes + tile * kRows * C::P;
-      const int bytes = rows * C::P;
-      for (int q = lt; q < bytes / 16; q += 128)
-        reinterpret_cast<uint4*>(sRec)[q] = __ldg(reinterpret_cast<const uint4*>(src) + q);
-      for (int q = (bytes / 16) * 16 + lt; q < bytes; q += 128) sRec[q] = src[q];
-      group_sync(g);
-    }
-    // unpack, gather, split into the A tiles
-    uint32_t w[(C::P + 3) / 4 + 1];
-#pragma unroll
-    for (int q = 0; q < (C::P + 3) / 4 + 1; ++q) w[q] = 0u;
-    if (lt < rows) {
-      const uint8_t* rec = sRec + lt * C::P;
-      if constexpr (C::P % 4 == 0) {
-#pragma unroll
-        for (int q = 0; q < C::P / 4; ++q) w[q] = reinterpret_cast<const uint32_t*>(rec)[q];
-      } else if constexpr (C::P % 2 == 0) {
-#pragma unroll
-        for (int q = 0; q < C::P / 2; ++q)
-          w[q / 2] |= uint32_t(reinterpret_cast<const uint16_t*>(rec)[q]) << (16 * (q & 1));
-      } else {
-#pragma unroll
-        for (int q = 0; q < C::P; ++q) w[q / 4] |= uint32_t(rec[q]) << (8 * (q & 3));
-      }
-    }
-    // gather codewords and write the A tiles one 16-byte chunk (8 coordinates) at a time
-    constexpr int NCH = (DP + 7) / 8;
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
-      const int j0 = (8 * c) / K;
-      const int j1 = ((8 * c + 7) / K < C::M - 1) ? (8 * c + 7) / K : C::M - 1;
-#pragma unroll
-      for (int j = j0; j <= j1; ++j) {
-        const int off = j * B;
-        uint32_t id = w[off / 32] >> (off % 32);
-        if ((off % 32) + B > 32) id |= w[off / 32 + 1] << (32 - off % 32);
-        id &= (1u << B) - 1u;
-        uint32_t eh[2], el[2];  // hi / lo half2 words of the codeword (up to 4 halves each)
-        if constexpr (K == 2) {
-          const uint2 e = *reinterpret_cast<const uint2*>(sCb + id * 8);
-          eh[0] = e.x; eh[1] = 0u; el[0] = e.y; el[1] = 0u;
-        } else {
-          const uint4 e = *reinterpret_cast<const uint4*>(sCb + id * 16);
-          eh[0] = e.x; eh[1] = e.y; el[0] = e.z; el[1] = e.w;
-        }
-#pragma unroll
-        for (int a = 0; a < K; ++a) {
-          const int hp = K * j + a;
-          if (hp >= 8 * c && hp < 8 * c + 8) {
-            const int q = hp - 8 * c;
-            const uint32_t hh = (eh[a >> 1] >> (16 * (a & 1))) & 0xFFFFu;
-            const uint32_t ll = (el[a >> 1] >> (16 * (a & 1))) & 0xFFFFu;
-            hw[q >> 1] |= hh << (16 * (q & 1));
-            lw[q >> 1] |= ll << (16 * (q & 1));
-          }
-        }
-      }
-      if (c < 8) {
-        *reinterpret_cast<uint4*>(sAh + ptx::sw128_offset(lt, 8 * c)) =
-            make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(sAl + ptx::sw128_offset(lt, 8 * c)) =
-            make_uint4(lw[0], lw[1], lw[2], lw[3]);
-      } else {
-        *reinterpret_cast<uint4*>(sAh + kRows * 128 + ptx::noswz16_offset(lt, 0)) =
-            make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(sAl + kRows * 128 + ptx::noswz16_offset(lt, 0)) =
-            make_uint4(lw[0], lw[1], lw[2], lw[3]);
-      }
-    }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    group_sync(g);  // A tiles written; this tile's records no longer read
-    if (lt == 0) {
-      if (tile + 2 * stride < n_full) issue_rec(tile + 2 * stride, s);
-      ptx::tc_fence_after();
-#pragma unroll
-      for (int ks = 0; ks < C::KSTEPS; ++ks) {
-        uint64_t ad, bd;
-        if (ks < 4) {
-          ad = ptx::sdesc_kmajor_sw128(aH + ks * 32);
-          bd = ptx::sdesc_kmajor_sw128(bA + ks * 32);
-        } else {
-          ad = ptx::sdesc_kmajor_noswz(aH + kRows * 128, 128, 256);
-          bd = ptx::sdesc_kmajor_noswz(bA + 128 * 128, 128, 256);
-        }
-        ptx::umma_f16(acc, ad, bd, idesc128, ks > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int ks = 0; ks < C::KSTEPS; ++ks) {
-        uint64_t ad, bd;
-        if (ks < 4) {
-          ad = ptx::sdesc_kmajor_sw128(aL + ks * 32);
-          bd = ptx::sdesc_kmajor_sw128(bA + ks * 32);
-        } else {
-          ad = ptx::sdesc_kmajor_noswz(aL + kRows * 128, 128, 256);
-          bd = ptx::sdesc_kmajor_noswz(bA + 128 * 128, 128, 256);
-        }
-        ptx::umma_f16(acc + 64, ad, bd, idesc64, 1u);
-      }
-      ptx::umma_commit(mma_bar);
-    }
-    const bool ok = ptx::mbar_wait(mma_bar, i & 1);
-    ptx::tc_fence_after();
-    if (!ok) sFlag[g] = 1;
-    const int64_t row = tile * kRows + lt;
-#pragma unroll
-    for (int c = 0; c < 64; c += 16) {
-      uint32_t h[16], l[16];
-      ptx::tmem_ld16(acc + lane_base + c, h);
-      ptx::tmem_ld16(acc + lane_base + 64 + c, l);
-      ptx::tmem_wait_ld();
-      float v[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        v[e] = nu * fmaf(__uint_as_float(l[e]), kLoScale, __uint_as_float(h[e]));
-      if (lt < rows) {
-        if constexpr (OUT_F16) {
-          uint32_t o[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const __half2 hv2 = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
-            o[e] = *reinterpret_cast<const uint32_t*>(&hv2);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + row * 64 + c);
-          dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-          dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-        } else {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.y) + row * 64 + c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-        }
-      }
-    }
-    ptx::tc_fence_before();
-    group_sync(g);  // A tiles, records and TMEM free for the next tile
-    if (*(volatile int*)&sFlag[g]) break;
-  }
-  ptx::tc_fence_before();
-  __syncthreads();
-  if (tid == 0 && (sFlag[0] | sFlag[1] | sFlag[2] | sFlag[3]))
-    atomicAdd(&g_fq_wait_timeouts, 1u);
-  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
-}
-
 // ---- host side --------------------------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
@@ -911,33 +593,6 @@ cudaError_t launch_enc(const void* x, int64_t n, const EncParams& p, cudaStream_
   return launch_enc_kernel<K, DP, B, false>(x, n, p, st);
 }
 
-template <int K, int DP, int B, bool F16>
-cudaError_t launch_dec(const DecParams& p, cudaStream_t st) {
-  using C = DecCfg<K, DP, B, F16>;
-  auto kern = decode_d64_kernel<K, DP, B, F16>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  const int64_t tiles = (p.n + kRows - 1) / kRows;
-  const int64_t ctas = std::min<int64_t>((tiles + kDecGroups - 1) / kDecGroups, sm_count());
-  kern<<<(int)ctas, kDecThreads, C::SMEM, st>>>(p);
-  return cudaGetLastError();
-}
-
-template <int K, int DP, bool F16>
-cudaError_t dec_dispatch_B(int B, const DecParams& p, cudaStream_t st) {
-  switch (B) {
-    case 1: return launch_dec<K, DP, 1, F16>(p, st);
-    case 2: return launch_dec<K, DP, 2, F16>(p, st);
-    case 3: return launch_dec<K, DP, 3, F16>(p, st);
-    case 4: return launch_dec<K, DP, 4, F16>(p, st);
-    case 5: return launch_dec<K, DP, 5, F16>(p, st);
-    case 6: return launch_dec<K, DP, 6, F16>(p, st);
-    case 7: return launch_dec<K, DP, 7, F16>(p, st);
-    case 8: return launch_dec<K, DP, 8, F16>(p, st);
-  }
-  return cudaErrorNotSupported;
-}
-
 template <int K, int DP>
 cudaError_t dispatch_B(int B, const void* x, int64_t n, const EncParams& p, cudaStream_t st) {
   switch (B) {
@@ -980,36 +635,6 @@ cudaError_t launch_encode(const void* x, fq_dtype, int64_t n, const Shape& s, co
     case 2: return dispatch_B<2, 64>(s.B, x, n, p, st);
     case 3: return dispatch_B<3, 66>(s.B, x, n, p, st);
     case 4: return dispatch_B<4, 64>(s.B, x, n, p, st);
-  }
-  return cudaErrorNotSupported;
-}
-
-bool decode_supported(fq_dtype yt, const Shape& s, const void* codes, const void* norms,
-                      const void* y) {
-  (void)norms;
-  if (s.d != 64 || s.N > 256 || s.k < 2 || s.k > 4) return false;
-  if ((reinterpret_cast<uintptr_t>(y) & 15) || (reinterpret_cast<uintptr_t>(codes) & 15))
-    return false;
-  (void)yt;
-  return is_sm100();
-}
-
-cudaError_t launch_decode(const uint8_t* codes, const uint16_t* norms, int64_t n,
-                          const Shape& s, const float* rot, const float* cb, void* y,
-                          fq_dtype yt, cudaStream_t st) {
-  DecParams p;
-  p.n = n;
-  p.N = s.N;
-  p.rot = rot;
-  p.cb = cb;
-  p.codes = codes;
-  p.norms = norms;
-  p.y = y;
-  const bool f16 = yt == FQ_F16;
-  switch (s.k) {
-    case 2: return f16 ? dec_dispatch_B<2, 64, true>(s.B, p, st) : dec_dispatch_B<2, 64, false>(s.B, p, st);
-    case 3: return f16 ? dec_dispatch_B<3, 66, true>(s.B, p, st) : dec_dispatch_B<3, 66, false>(s.B, p, st);
-    case 4: return f16 ? dec_dispatch_B<4, 64, true>(s.B, p, st) : dec_dispatch_B<4, 64, false>(s.B, p, st);
   }
   return cudaErrorNotSupported;
 }
