@@ -79,7 +79,8 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []   # (arrival time, line)
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
@@ -89,15 +90,20 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            deadline = time.time() + 5.0  # the sampler is running before the region starts
+            while not self.lines and time.time() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
         except (OSError, FileNotFoundError):
             self.proc = None
+        self.t0 = time.time()
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
     def __exit__(self, *a):
+        self.t1 = time.time()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -108,7 +114,9 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.lines:
+            if self.t0 is not None and not (self.t0 <= ts <= self.t1 + 0.1):
+                continue  # only samples taken while the timed region ran
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 7:
                 continue
@@ -255,32 +263,40 @@ def run_gpu(args):
         torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
-    # warm-up
-    for i in range(args.warmup):
-        c = i % copies
-        for lab, kind, ab, eb, fn in codec_launches(fq, shape, xs, ys, states, c, (c - 1) % copies):
+    # The timed region replays CUDA graphs of the step's C-ABI calls (one graph per input copy):
+    # the kernels, arguments and order are those of the eager calls, without the host-side
+    # launch latency between them.
+    side = torch.cuda.Stream(device)
+    side.wait_stream(stream)
+
+    def capture(fns):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for fn in fns:
+                    fn()
+        return g
+
+    for c in range(copies):  # one eager pass (tables, attributes) before capture
+        for *_, fn in codec_launches(fq, shape, xs, ys, states, c, (c - 1) % copies):
             fn()
-        if attn_launch:
-            attn_launch(i % 4)
+    torch.cuda.synchronize()
+    step_graphs = [capture([fn for *_, fn in codec_launches(fq, shape, xs, ys, states, c,
+                                                             (c - 1) % copies)])
+                   for c in range(copies)]
+    meta = [(lab, kind, ab, eb) for lab, kind, ab, eb, _ in
+            codec_launches(fq, shape, xs, ys, states, 0, copies - 1)]
+    torch.cuda.synchronize()
+    for i in range(args.warmup):
+        step_graphs[i % copies].replay()
     barrier()
-    # timed region: K steps, per-launch events on the launching stream
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(n_launch)] for _ in range(args.steps)]
-    meta = None
     with ClockSampler(local) as clk:
         barrier()
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record(stream)
         for i in range(args.steps):
-            c = i % copies
-            launches = list(codec_launches(fq, shape, xs, ys, states, c, (c - 1) % copies))
-            if meta is None:
-                meta = [(lab, kind, ab, eb) for lab, kind, ab, eb, _ in launches]
-            for j, (_, _, _, _, fn) in enumerate(launches):
-                ev[i][j][0].record(stream)
-                fn()
-                ev[i][j][1].record(stream)
+            step_graphs[i % copies].replay()
         t_end.record(stream)
         barrier()
     total_ms = t_start.elapsed_time(t_end)
@@ -288,25 +304,37 @@ def run_gpu(args):
         t = torch.tensor([total_ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
+    # per-kernel device time: a graph of every launch of one kind over all copies, replayed
     per = {}
-    for i in range(args.steps):
-        for j, (lab, kind, ab, eb) in enumerate(meta):
-            ms = ev[i][j][0].elapsed_time(ev[i][j][1])
-            s = per.setdefault(lab, {"ms": 0.0, "launches": 0, "alg_bytes": ab, "kind": kind,
-                                     "eq_bytes": 0})
-            s["ms"] += ms
-            s["launches"] += 1
+    reps = max(5, min(50, args.steps // copies))
+    for lab in dict.fromkeys(m[0] for m in meta):
+        fns = [fn for c in range(copies) for l, *_, fn in
+               codec_launches(fq, shape, xs, ys, states, c, (c - 1) % copies) if l == lab]
+        g = capture(fns)
+        g.replay()
+        barrier()
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        k1.record(stream)
+        barrier()
+        ms = k0.elapsed_time(k1) / (reps * len(fns))
+        ab, kind = next((m[2], m[1]) for m in meta if m[0] == lab)
+        per_step = sum(1 for m in meta if m[0] == lab)
+        per[lab] = {"ms": ms, "per_step": per_step, "alg_bytes": ab, "kind": kind}
+        del g
     step_eq = sum(eb for _, _, _, eb in meta)
     value = world * step_eq * args.steps / (total_ms * 1e-3) / 1e9
     hbm, hbm_src = peaks()
-    dom_lab = max(per, key=lambda k: per[k]["ms"])
+    dom_lab = max(per, key=lambda k: per[k]["ms"] * per[k]["per_step"])
     dom = per[dom_lab]
-    avg_ms = dom["ms"] / dom["launches"]
-    achieved = dom["alg_bytes"] / (avg_ms * 1e-3) / 1e9
-    kernels = {lab: {"avg_us": round(1e3 * s["ms"] / s["launches"], 2),
-                     "GBps_alg": round(s["alg_bytes"] / (s["ms"] / s["launches"] * 1e-3) / 1e9, 1),
-                     "share": round(s["ms"] / sum(v["ms"] for v in per.values()), 3)}
-               for lab, s in per.items()}
+    achieved = dom["alg_bytes"] / (dom["ms"] * 1e-3) / 1e9
+    tot_share = sum(v["ms"] * v["per_step"] for v in per.values())
+    kernels = {lab: {"avg_us": round(1e3 * s_["ms"], 2),
+                     "GBps_alg": round(s_["alg_bytes"] / (s_["ms"] * 1e-3) / 1e9, 1),
+                     "share": round(s_["ms"] * s_["per_step"] / tot_share, 3)}
+               for lab, s_ in per.items()}
     result = {
         "metric": "KV encode/decode GB/s (fp16-equiv) & % of roofline; fused attn us/step",
         "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -316,7 +344,8 @@ def run_gpu(args):
         "config": {"workload": w.name, "vectors_per_gpu": shape.n, "d": shape.d,
                    "rates": [r.label for r in w.rates], "decode_out": "fp16",
                    "l2": f"inputs rotate over {copies} copies (>= 2x L2 between reuses)",
-                   "step": "encode K,V + decode K,V per rate"},
+                   "step": "encode K,V + decode K,V per rate",
+                   "launch": "CUDA graph replay of the step's C-ABI calls"},
         "roofline": {"bound": "hbm", "kernel": dom_lab, "achieved": round(achieved, 1),
                      "peak": hbm, "peak_source": hbm_src, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": profiled_traffic(dom_lab),
@@ -325,25 +354,33 @@ def run_gpu(args):
         "gpu_launches": None,
         "clocks": clk.summary(),
     }
-    launches_per_step = sum(1 for _ in meta)
+    launches_per_step = len(meta)
     gpu_launches = launches_per_step * args.steps
     # fused attention step
     if attn_launch:
-        reps = max(20, args.steps // 10)
+        for c in range(4):
+            attn_launch(c)
+        torch.cuda.synchronize()
+        agraphs = [capture([lambda c=c: attn_launch(c)]) for c in range(4)]
+        areps = max(20, args.steps // 10)
+        for i in range(4):
+            agraphs[i].replay()
         barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for i in range(reps):
-            attn_launch(i % 4)
+        for i in range(areps):
+            agraphs[i % 4].replay()
         a1.record(stream)
         barrier()
-        us = a0.elapsed_time(a1) * 1e3 / reps
+        us = a0.elapsed_time(a1) * 1e3 / areps
         result["attn"] = {"workload": wl.ATTN.name, "us_per_step": round(us, 2),
                           "bytes_per_step": attn_bytes,
                           "roofline": {"bound": "hbm", "achieved": round(attn_bytes / (us * 1e-6) / 1e9, 1),
                                        "peak": hbm, "unit": "GB/s",
                                        "frac": round(attn_bytes / (us * 1e-6) / 1e9 / hbm, 4)},
                           "launches_per_step": 2}
+        del agraphs
+    del step_graphs
     result["gpu_launches"] = gpu_launches
     # end to end through the public API with pinned host buffers
     if not args.no_e2e:
@@ -465,7 +502,7 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="fibquant", choices=["fibquant", "reference"])
     ap.add_argument("--workload", default="gpt2", choices=list(WORKLOADS))

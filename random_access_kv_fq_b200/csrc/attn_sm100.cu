@@ -33,7 +33,7 @@
 
 namespace fq {
 
-extern __device__ unsigned int g_fq_wait_timeouts;
+__device__ unsigned int g_fq_wait_timeouts = 0;  // CTAs whose bounded waits gave up
 
 namespace attn100 {
 namespace {

@@ -36,7 +36,7 @@
 namespace fq {
 namespace sm100 {
 
-extern __device__ unsigned int g_fq_wait_timeouts;
+
 
 namespace {
 
