@@ -62,6 +62,7 @@ struct Cfg {
   // tensor memory columns: key A operand (hi | lo), scores, value accumulators
   static constexpr int C_AH = 0, C_AL = 32, C_D1 = 64, C_D2 = C_D1 + N1, C_DV = C_D2 + N2;
   static constexpr int TMEM_COLS = (C_DV + NVM <= 128) ? 128 : 256;
+  static constexpr int MIN_CTAS = (TMEM_COLS == 128) ? 3 : 2;  // CTAs sharing an SM
   // value codeword table: 8 bank-private copies when small (conflict-free 16-byte lookups)
   static constexpr int VREP = (NV <= 64) ? 8 : 1;
   // one ring stage: key records, value records, key norms, value norms (each a 16-byte aligned
@@ -187,7 +188,8 @@ __device__ __forceinline__ void value_chunk(const uint4 (&e)[MV], bool hi, uint3
 }
 
 template <int G, int KB, int KV, int VB>
-__global__ void __launch_bounds__(kThr) attn_partial_sm100(AttnArgs a) {
+__global__ void __launch_bounds__(kThr, Cfg<G, KB, KV, VB>::MIN_CTAS)
+    attn_partial_sm100(AttnArgs a) {
   using C = Cfg<G, KB, KV, VB>;
   constexpr int PK = C::PK, PV = C::PV;
   extern __shared__ uint8_t smem_raw[];
@@ -262,7 +264,9 @@ __global__ void __launch_bounds__(kThr) attn_partial_sm100(AttnArgs a) {
   };
 
   // ---- set-up ----
-  int issued = 0;  // thread 0: tiles handed to the ring
+  // Single-thread work is spread over three warps so that no warp serialises all of it:
+  // thread 0 issues the score MMAs, thread 32 the bulk copies, thread 64 the value MMAs.
+  int issued = 0;  // thread 0 during set-up, then thread 32: tiles handed to the ring
   if (warp == 0) {
     ptx::tmem_alloc(sTmem, C::TMEM_COLS);
     ptx::tmem_relinquish();
@@ -280,10 +284,24 @@ __global__ void __launch_bounds__(kThr) attn_partial_sm100(AttnArgs a) {
   // Pi_K (rows padded to 65 floats) and the group's queries, staged in the value tile's space
   float* sRot = reinterpret_cast<float*>(sAV);
   float* sQf = sRot + 64 * 65;
-  for (int e = tid; e < 64 * 64; e += kThr) sRot[(e >> 6) * 65 + (e & 63)] = __ldg(a.rotK + e);
-  {
+  {  // loads issued eight at a time before their stores
+#pragma unroll 1
+    for (int i0 = 0; i0 < 64 * 64 / kThr; i0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it) v[it] = __ldg(a.rotK + tid + (i0 + it) * kThr);
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int e = tid + (i0 + it) * kThr;
+        sRot[(e >> 6) * 65 + (e & 63)] = v[it];
+      }
+    }
     const uint16_t* qg = a.q + ((size_t)b * a.Hq + (size_t)g * G) * 64;
-    for (int e = tid; e < G * 64; e += kThr) sQf[e] = f16_bits_to_f32(qg[e]);
+    uint16_t qv[G * 64 / kThr];
+#pragma unroll
+    for (int it = 0; it < G * 64 / kThr; ++it) qv[it] = qg[tid + it * kThr];
+#pragma unroll
+    for (int it = 0; it < G * 64 / kThr; ++it) sQf[tid + it * kThr] = f16_bits_to_f32(qv[it]);
   }
   // key table: (hi0, hi1 | lo0, lo1) per codeword
   for (int c = tid; c < C::NK; c += kThr) {
@@ -335,6 +353,7 @@ __global__ void __launch_bounds__(kThr) attn_partial_sm100(AttnArgs a) {
   constexpr uint32_t idesc2 = ptx::idesc_f16_f32(128, C::N2);
   constexpr uint32_t idescv = ptx::idesc_f16_f32_amn(128, C::NVM);
   const uint32_t aQ = ptx::smem_u32(sQ), aV = ptx::smem_u32(sAV), aP = ptx::smem_u32(sP);
+  if (tid == 32) issued = kStages < n_tiles ? kStages : n_tiles;  // thread 0 issued these
   const float sc0 = a.scale * kLog2e;
   // this thread's (token tid) addresses in the swizzled tiles, per row / chunk class r = 0..7
   uint32_t p_off[8], av_off[8];
@@ -353,7 +372,7 @@ __global__ void __launch_bounds__(kThr) attn_partial_sm100(AttnArgs a) {
   }
   float sig = 0.f, inv_sig = 0.f;
   bool failed = false;
-  int last_k = -1, last_v = -1;  // thread 0: last committed score / value MMA (tile index)
+  int last_k = -1, last_v = -1;  // threads 0 / 64: last committed score / value MMA (tile)
 
   // weights w = p nu / sigma into the B tile: hi in row h, 2^12-scaled lo in row G + h
   auto write_weights = [&](const float (&pv)[G], float wn) {
@@ -425,17 +444,21 @@ __global__ void __launch_bounds__(kThr) attn_partial_sm100(AttnArgs a) {
     }
     if (tid == 0) {
       ptx::tc_fence_after();
+      // descriptor of the first K step; later steps add their byte offset / 16 to the start
+      // address field (the sums stay inside the 14-bit field for shared-memory addresses)
+      const uint64_t dq0 = ptx::sdesc_kmajor_sw128(aQ);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)  // + 32 B per K step
+        ptx::umma_f16_ts(tmem + C::C_D1, tmem + C::C_AH + 8 * ks, dq0 + 2 * ks, idesc1,
+                         ks > 0 ? 1u : 0u);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        ptx::umma_f16_ts(tmem + C::C_D1, tmem + C::C_AH + 8 * ks,
-                         ptx::sdesc_kmajor_sw128(aQ + ks * 32), idesc1, ks > 0 ? 1u : 0u);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        ptx::umma_f16_ts(tmem + C::C_D2, tmem + C::C_AL + 8 * ks,
-                         ptx::sdesc_kmajor_sw128(aQ + ks * 32), idesc2, ks > 0 ? 1u : 0u);
+        ptx::umma_f16_ts(tmem + C::C_D2, tmem + C::C_AL + 8 * ks, dq0 + 2 * ks, idesc2,
+                         ks > 0 ? 1u : 0u);
       ptx::umma_commit(bar_k);
       last_k = i;
-      if (issued < n_tiles) issue_tile(issued++);
+    } else if (tid == 32 && issued < n_tiles) {
+      issue_tile(issued++);
     }
 
     // ---- values: zhat^V_t (hi rows 0..63, lo rows 64..127) as column t of the MN-major A
@@ -571,25 +594,28 @@ __global__ void __launch_bounds__(kThr) attn_partial_sm100(AttnArgs a) {
         }
       }
     }
-    if (tid == 0) {
+    if (tid == 64) {
       ptx::tc_fence_after();
+      const uint64_t dv0 = ptx::sdesc_mnmajor_sw128(aV, 1024, 2048);
+      const uint64_t dp0 = ptx::sdesc_kmajor_sw128(aP);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        ptx::umma_f16(tmem + C::C_DV, ptx::sdesc_mnmajor_sw128(aV + ks * 4096, 1024, 2048),
-                      ptx::sdesc_kmajor_sw128(aP + (ks >> 2) * 4096 + (ks & 3) * 32), idescv,
-                      (i > 0 || ks > 0) ? 1u : 0u);
+      for (int ks = 0; ks < 8; ++ks)  // A: + 4096 B per step; B: + 4096 B per 4 steps, + 32 B
+        ptx::umma_f16(tmem + C::C_DV, dv0 + 256 * ks, dp0 + 256 * (ks >> 2) + 2 * (ks & 3),
+                      idescv, (i > 0 || ks > 0) ? 1u : 0u);
       ptx::umma_commit(bar_v);
       last_v = i;
     }
   }
 
   // ---- after a timed-out wait: let this CTA's own copies and MMAs in flight land (bounded)
-  if (tid == 0 && failed) {
-    for (int t = 0; t < issued; ++t)
-      if (t + kStages >= issued) ptx::mbar_wait(&full[t % kStages], (uint32_t)(t / kStages) & 1u);
-    if (last_k >= 0) ptx::mbar_wait(bar_k, (uint32_t)last_k & 1u);
-    if (last_v >= 0) ptx::mbar_wait(bar_v, (uint32_t)last_v & 1u);
+  if (failed) {
+    if (tid == 32)
+      for (int t = issued - kStages < 0 ? 0 : issued - kStages; t < issued; ++t)
+        ptx::mbar_wait(&full[t % kStages], (uint32_t)(t / kStages) & 1u);
+    if (tid == 0 && last_k >= 0) ptx::mbar_wait(bar_k, (uint32_t)last_k & 1u);
+    if (tid == 64 && last_v >= 0) ptx::mbar_wait(bar_v, (uint32_t)last_v & 1u);
   }
+  __syncwarp();
 
   // ---- partials of this split: (m, l, acc[d'_V]) per head, acc scaled back by sigma
   if (!failed && !ptx::mbar_wait(bar_v, (uint32_t)(n_tiles - 1) & 1u)) failed = true;
