@@ -1,4 +1,4 @@
-// sm_100a fast paths of fq_encode / fq_decode (declarations; see codec_sm100.cu).
+// sm_100a fast paths of fq_encode / fq_decode (encode_sm100.cu, encode_large_sm100.cu, decode_sm100.cu).
 #pragma once
 
 #include "fq_internal.h"
@@ -12,6 +12,13 @@ bool encode_supported(fq_dtype xt, const Shape& s, const void* x, const void* co
 cudaError_t launch_encode(const void* x, fq_dtype xt, int64_t n, const Shape& s,
                           const float* rot, const float* cb, uint8_t* codes, uint16_t* norms,
                           const void* index, cudaStream_t st);
+
+// Large codebooks (d = 128, k = 4, N = 512 .. 4096, no index): tensor-core brute force.
+bool encode_large_supported(fq_dtype xt, const Shape& s, const void* x, const void* codes,
+                            const float* cb, const void* index);
+cudaError_t launch_encode_large(const void* x, int64_t n, const Shape& s, const float* rot,
+                                const float* cb, uint8_t* codes, uint16_t* norms,
+                                cudaStream_t st);
 
 bool decode_supported(fq_dtype yt, const Shape& s, const void* codes, const void* norms,
                       const void* y);

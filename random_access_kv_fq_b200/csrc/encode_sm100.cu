@@ -90,10 +90,6 @@ __device__ __forceinline__ float sq2_acc(uint32_t hw, float acc) {
   return acc;
 }
 
-__device__ __forceinline__ void pipe_sync(int pipe) {
-  asm volatile("bar.sync %0, %1;" ::"r"(pipe + 1), "r"(128) : "memory");
-}
-
 // ---- nearest-codeword search policies ------------------------------------------------------
 // Scores are 1 + |c|^2 - 2 z.c: the squared distance minus |z|^2 (common to all candidates)
 // plus a constant.  Candidates are scanned in increasing index order with a strict less-than,

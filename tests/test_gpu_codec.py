@@ -224,3 +224,25 @@ def test_fast_and_generic_paths_meet_parity_on_the_same_rows(dp, k, N):
         results.append(gidx)
     diff = results[0] != results[1]
     assert not (diff & (enc.gap > par.NEAR_TIE_GAP)).any()
+
+
+@pytest.mark.parametrize("N", [512, 1024, 2048, 4096])
+def test_large_codebook_tensor_core_search(N):
+    """d = 128, k = 4, N = 512 .. 4096 without an index runs the tensor-core brute-force search
+    with fp32 re-ranking of near ties; indices must match the oracle's brute force (ties to the
+    lowest index).  N < 4096 uses unit-ball random codebooks (the search does not depend on
+    the codebook being Lloyd-optimal)."""
+    d, k = 128, 4
+    rot = tables.rotation(d, wl.ROT_SEED_K)
+    if N == 4096:
+        cb = tables.codebook(d, k, N)
+    else:
+        rng = np.random.default_rng(N)
+        u = rng.standard_normal((N, k))
+        u /= np.linalg.norm(u, axis=1, keepdims=True)
+        r = rng.beta(k / 2, (d - k) / 2, size=(N, 1)) ** 0.5
+        cb = (u * r).astype(np.float32)
+    x = wl.gaussian_rows(1000, d, seed=N, sigma=1.0)
+    x[7] = 0  # zero vector
+    x[8] = x[9]  # duplicate rows
+    run_codec(x, rot, cb, wl.Rate(k, N, "brute"), d)
