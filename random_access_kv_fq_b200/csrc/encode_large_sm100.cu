@@ -10,20 +10,22 @@
 //   A row  (block z)      [ z_hi(4) | z_hi(4)  | z_res(4) | 1       | 1        | 0 0 ]
 //   B row  (codeword n)   [ a_hi(4) | a_res(4) | a_hi(4)  | cc_hi   | cc_res   | 0 0 ]
 // with a = -2 c_n, cc = |c_n|^2 + 1, x_res = fp16(x - x_hi); the dropped z_res . a_res term is
-// ~2^-22 of the score.  The scan keeps, per quarter of the codebook, the two chunks with the
-// lowest approximate minima; every chunk whose minimum lies within kTie of the overall best is
-// then re-scored with exact fp32 squared distances to the block (from the fp32 codebook): the
-// lower distance wins, the lower index on equality, as in the oracle.
+// ~2^-22 of the score.  The scan keeps, per quarter of the codebook, the two 8-codeword groups
+// with the lowest approximate minima; every such group whose minimum lies within kTie of the
+// overall best is then re-scored with exact fp32 squared distances to the block (from the fp32
+// codebook): the lower distance wins, the lower index on equality, as in the oracle.
 //
 // One persistent CTA per SM, 128-vector tiles, 17 warps:
 //   warps 0-15  four warpgroups; warpgroup 0 (one thread per vector) loads x into tensor memory,
 //               computes nu and, per block, the A operand, and resolves the block's codeword;
 //               every warpgroup scans one quarter (32 scores) of each 128-codeword chunk:
-//               a minimum tree and a branch-free update of the best and second-best chunk
-//   warp 16     issues the rotation MMA and the chunk MMAs (two score buffers in tensor memory,
-//               so that the next chunk is computed while one is scanned)
-// Tensor memory: columns 0..255 rotation (hi | lo), 256..511 two 128-column score buffers (the
-// first also stages x during the rotation).
+//               a minimum tree down to four 8-codeword groups and a branch-free update of
+//               the best and runner-up group; after each block it re-scores those groups
+//   warp 16     issues the rotation MMA and the chunk MMAs (three score buffers in tensor
+//               memory, so that two chunks are computed ahead of the one being scanned)
+// Tensor memory: columns 0..255 rotation accumulators (hi | lo), combined once per tile into
+// fp32 z in columns 0..127; 128..511 three 128-column score buffers (the second also stages x
+// during the rotation).
 #include <cstdint>
 
 #include <cuda.h>
@@ -43,7 +45,8 @@ constexpr int kThreadsL = kScanThreads + 32;
 constexpr int kDL = 128;                  // d = d'
 constexpr int kML = 32;                   // blocks per vector (k = 4)
 constexpr int kChunk = 128;               // codewords per MMA
-constexpr int kBufs = 2;                  // score buffers in tensor memory (128 columns each)
+constexpr int kBufs = 3;                  // score buffers in tensor memory (128 columns each)
+constexpr uint32_t kTmScore = 128;        // first score buffer column
 constexpr int kPer = kChunk / 4;          // scores of a chunk per scanning warpgroup
 constexpr float kLoScaleL = 1.0f / 4096.0f;
 constexpr float kTie = 1.0f / 8192.0f;    // approximate-score band re-ranked exactly
@@ -77,13 +80,13 @@ struct LParams {
 
 __device__ __forceinline__ uint32_t h2u_l(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
-// Bounded wait (about 2^18 suspensions of <= 4 us, ~1 s) that gives up early when another
-// role raised the abort flag.  Waiting threads are suspended in the barrier instead of polling,
-// which keeps the shared-memory pipe free for the tensor cores' operand reads.
+// Bounded wait (at most 2^22 polls, well under a second) that gives up early when another role
+// raised the abort flag.  One lane per warp polls with the non-blocking test, so a completed
+// phase is seen at once.
 __device__ __forceinline__ bool wait_l(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  for (uint32_t it = 0; it < (ptx::kSpinLimit >> 2); ++it) {
-    if (ptx::mbar_try_sleep(bar, parity, 4000u)) return true;
-    if (*abort) return false;
+  for (uint32_t it = 0; it < (ptx::kSpinLimit << 2); ++it) {
+    if (ptx::mbar_test(bar, parity)) return true;
+    if ((it & 63u) == 63u && *abort) return false;
   }
   *abort = 1;
   return false;
@@ -127,8 +130,8 @@ __global__ void __launch_bounds__(kThreadsL, 1) encode_large_kernel(LParams p) {
   uint64_t* x_ready = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // x staged (4 warps)
   uint64_t* rot_done = x_ready + 1;                                   // rotation MMA done
   uint64_t* a_ready = rot_done + 1;                                   // [2] A tile built (4 warps)
-  uint64_t* full = a_ready + 2;                                       // [4] scores ready
-  uint64_t* empty = full + kBufs;                                     // [4] scores read (16 warps)
+  uint64_t* full = a_ready + 2;                                       // [3] scores ready
+  uint64_t* empty = full + kBufs;                                     // [3] scores read (16 warps)
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(empty + kBufs);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
   uint32_t* sRec = reinterpret_cast<uint32_t*>(smem + C::OFF_REC);
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(kThreadsL, 1) encode_large_kernel(LParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *sTmem;
-  constexpr uint32_t TM_X = 256;  // x staging (first score buffer)
+  constexpr uint32_t TM_X = 256;  // x staging (second score buffer)
 
   if (warp == 16) {
     // ---- MMA issuer: rotation of each tile, then CHUNKS score MMAs per block ----
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(kThreadsL, 1) encode_large_kernel(LParams p) {
             const int buf = g % kBufs;
             if (g >= kBufs && !(ok = wait_l(&empty[buf], ((g / kBufs) - 1) & 1u, sAbort))) break;
             ptx::tc_fence_after();
-            ptx::umma_f16(tmem + 256 + kChunk * buf, ad,
+            ptx::umma_f16(tmem + kTmScore + kChunk * buf, ad,
                           ptx::sdesc_kmajor_noswz(cbA + kChunk * 32 * c, 128, 256), idesc_s, 0u);
             ptx::umma_commit(&full[buf]);
           }
@@ -256,20 +259,16 @@ __global__ void __launch_bounds__(kThreadsL, 1) encode_large_kernel(LParams p) {
   } else {
     // ---- scanners (warpgroup wg: columns 32 wg .. 32 wg + 31 of every chunk) ----
     uint32_t g = 0;
-    float nu = 0.f, rinv = 0.f, zc[4] = {0.f, 0.f, 0.f, 0.f}, zn[4] = {0.f, 0.f, 0.f, 0.f};
+    float nu = 0.f, rinv = 0.f;
     bool aborted = false;
     // A tile of block j for this row (warpgroup 0): z from the rotation in tensor memory
-    auto build_a = [&](int j, float (&z)[4]) {
-      uint32_t h[4], l[4];
-      ptx::tmem_ld4(tmem + lane_base + 4 * j, h);
-      ptx::tmem_ld4(tmem + lane_base + 128 + 4 * j, l);
+    auto build_a = [&](int j) {
+      uint32_t zw[4];
+      ptx::tmem_ld4(tmem + lane_base + 4 * j, zw);
       ptx::tmem_wait_ld();
       __half zh[4], zr[4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        z[a] = fmaf(__uint_as_float(l[a]), kLoScaleL * rinv, __uint_as_float(h[a]) * rinv);
-        split_hr(z[a], zh[a], zr[a]);
-      }
+      for (int a = 0; a < 4; ++a) split_hr(__uint_as_float(zw[a]), zh[a], zr[a]);
       const __half one = __float2half_rn(1.f), z0 = __float2half_rn(0.f);
       uint8_t* r0 = sA + (j & 1) * 4096 + ptx::noswz16_offset((uint32_t)row, 0);
       const uint32_t w0 = h2u_l(__halves2half2(zh[0], zh[1])), w1 = h2u_l(__halves2half2(zh[2], zh[3]));
@@ -287,39 +286,32 @@ __global__ void __launch_bounds__(kThreadsL, 1) encode_large_kernel(LParams p) {
       bool fail = false;
       if (wg == 0) {
         // x row -> tensor memory (A operand of the rotation), nu from the exact fp16 squares
-        uint32_t xw[64];
-        if (vrow < p.n) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.x + vrow * kDL);
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const uint4 v = __ldg(src + q);
-            xw[4 * q] = v.x; xw[4 * q + 1] = v.y; xw[4 * q + 2] = v.z; xw[4 * q + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 64; ++q) xw[q] = 0u;
-        }
+        // in four 16-word pieces
+        const uint4* src = reinterpret_cast<const uint4*>(p.x + vrow * kDL);
         float part[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float a2 = 0.f;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xw[8 * c + q]));
-            a2 = fmaf(f.x, f.x, a2);
-            a2 = fmaf(f.y, f.y, a2);
-          }
-          part[c] = a2;
-        }
-        nu = sqrtf(((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7])));
-        rinv = nu > 0.f ? __frcp_rn(nu) : 0.f;
-#pragma unroll
+#pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           uint32_t r16[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r16[e] = xw[16 * q + e];
+          for (int e = 0; e < 4; ++e) {
+            const uint4 v = vrow < p.n ? __ldg(src + 4 * q + e) : make_uint4(0u, 0u, 0u, 0u);
+            r16[4 * e] = v.x; r16[4 * e + 1] = v.y; r16[4 * e + 2] = v.z; r16[4 * e + 3] = v.w;
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float a2 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r16[8 * h + e]));
+              a2 = fmaf(f.x, f.x, a2);
+              a2 = fmaf(f.y, f.y, a2);
+            }
+            part[2 * q + h] = a2;
+          }
           ptx::tmem_st16(tmem + lane_base + TM_X + 16 * q, r16);
         }
+        nu = sqrtf(((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7])));
+        rinv = nu > 0.f ? __frcp_rn(nu) : 0.f;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
@@ -327,86 +319,139 @@ __global__ void __launch_bounds__(kThreadsL, 1) encode_large_kernel(LParams p) {
         fail = !wait_l(rot_done, (uint32_t)i & 1u, sAbort);
         fail = __any_sync(0xffffffffu, fail);
         ptx::tc_fence_after();
-        if (!fail) build_a(0, zn);
+        if (!fail) {
+          // z = (D_hi + 2^-12 D_lo) / nu into columns 0..127 (frees 128..255 for scores)
+#pragma unroll 1
+          for (int q = 0; q < 16; ++q) {
+            uint32_t h[8], l[8];
+            ptx::tmem_ld8(tmem + lane_base + 8 * q, h);
+            ptx::tmem_ld8(tmem + lane_base + 128 + 8 * q, l);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              h[e] = __float_as_uint(
+                  fmaf(__uint_as_float(l[e]), kLoScaleL * rinv, __uint_as_float(h[e]) * rinv));
+            ptx::tmem_st8(tmem + lane_base + 8 * q, h);
+          }
+          ptx::tmem_wait_st();
+          build_a(0);
+        }
       }
       for (int j = 0; j < kML; ++j) {
-        if (wg == 0) {
-#pragma unroll
-          for (int a = 0; a < 4; ++a) zc[a] = zn[a];
-          if (j + 1 < kML && !fail) build_a(j + 1, zn);
-        }
-        // Chunk minima of this warpgroup's quarter: the best and the second-best chunk (by
-        // their minima) are kept with selects only; the codewords inside them are resolved
-        // exactly once the block is done.
+        if (wg == 0 && j + 1 < kML && !fail) build_a(j + 1);
+        // Per chunk, this warpgroup's 32 scores reduce to four minima of 8-codeword groups.
+        // The best group (bg) and the runner-up group (sg: the best group of another chunk, or
+        // the second group of the best chunk) are kept with selects only, as group ids
+        // 4 * chunk + group; the codewords inside them are re-scored exactly after the block.
         float best = INFINITY, second = INFINITY;
-        int bc = 0, sc = -1;
+        int bg = 0, sg = -1;
+#pragma unroll 1
         for (int c = 0; c < C::CHUNKS; ++c, ++g) {
-          const int buf = g % kBufs;
-          if (!fail) fail = !wait_l(&full[buf], (g / kBufs) & 1u, sAbort);
-          fail = __any_sync(0xffffffffu, fail);
+          const uint32_t buf = g % kBufs;
+          bool ok = true;  // one lane polls the barrier for the warp
+          if (lane == 0 && !fail) ok = wait_l(&full[buf], (g / kBufs) & 1u, sAbort);
+          fail = fail || __shfl_sync(0xffffffffu, (int)ok, 0) == 0;
+          __syncwarp();
           if (fail) continue;
           ptx::tc_fence_after();
           uint32_t v[kPer];
-          ptx::tmem_ld_cols<0, kPer>(tmem + lane_base + 256 + kChunk * buf + kPer * wg, v);
+          ptx::tmem_ld_cols<0, kPer>(tmem + lane_base + kTmScore + kChunk * buf + kPer * wg, v);
           ptx::tmem_wait_ld();
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&empty[buf]);
-          float m[kPer / 2];
+          static_assert(kPer == 32, "four 8-column groups per chunk quarter");
+          float m2[16], m4[8];
 #pragma unroll
-          for (int q = 0; q < kPer / 2; ++q)
-            m[q] = fminf(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
+          for (int q = 0; q < 16; ++q)
+            m2[q] = fminf(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
 #pragma unroll
-          for (int w = kPer / 4; w >= 1; w >>= 1)
-#pragma unroll
-            for (int q = 0; q < w; ++q) m[q] = fminf(m[q], m[q + w]);
-          const float mv = m[0];
-          const bool nb = mv < best;               // earlier chunk kept on equal minima
+          for (int q = 0; q < 8; ++q) m4[q] = fminf(m2[2 * q], m2[2 * q + 1]);
+          // minima of the groups of columns 8k .. 8k + 7
+          const float o0 = fminf(m4[0], m4[1]), o1 = fminf(m4[2], m4[3]);
+          const float o2 = fminf(m4[4], m4[5]), o3 = fminf(m4[6], m4[7]);
+          const bool a01 = o1 < o0, a23 = o3 < o2;
+          const float w01 = a01 ? o1 : o0, l01 = a01 ? o0 : o1;
+          const float w23 = a23 ? o3 : o2, l23 = a23 ? o2 : o3;
+          const bool top = w23 < w01;
+          const float mv = top ? w23 : w01;
+          const int gid = top ? 2 + (int)a23 : (int)a01;
+          const float lt = top ? w01 : w23;  // loser of the final comparison
+          const int lid = top ? (int)a01 : 2 + (int)a23;
+          const float lw = top ? l23 : l01;  // loser inside the winning pair
+          const int wid = top ? 2 + (int)!a23 : (int)!a01;
+          const bool rl = lt <= lw;
+          const float rv = rl ? lt : lw;     // runner-up group of this chunk
+          const int rid = rl ? lid : wid;
+          const bool nb = mv < best;         // the earlier group is kept on equal minima
           const bool ns = !nb && mv < second;
-          second = nb ? best : (ns ? mv : second);
-          sc = nb ? bc : (ns ? c : sc);
+          const bool keep_old = best <= rv;  // on a new best: old best or this chunk's runner-up
+          second = nb ? (keep_old ? best : rv) : (ns ? mv : second);
+          sg = nb ? (keep_old ? bg : 4 * c + rid) : (ns ? 4 * c + gid : sg);
           best = nb ? mv : best;
-          bc = nb ? c : bc;
+          bg = nb ? 4 * c + gid : bg;
         }
-        sRes[((j & 1) * 4 + wg) * kRowsL + row] =
-            make_float4(best, __int_as_float(bc), second, __int_as_float(sc));
+        float4* mine = sRes + ((j & 1) * 4 + wg) * kRowsL + row;
+        *mine = make_float4(best, __int_as_float(bg), second, __int_as_float(sg));
         if (scan_sync_or(fail)) {
           aborted = true;
           break;
         }
-        if (wg == 0) {
-          // Every codeword that can be the nearest lies in a chunk whose approximate minimum
-          // is within kTie of the global approximate best (the approximation errs by ~2^-20):
-          // such chunks (the best and second-best chunk of each quarter) are re-scored with
-          // exact fp32 squared distances; the lower distance wins, the lower index on equality.
+        // Every codeword that can be the nearest lies in a group whose approximate minimum is
+        // within kTie of the overall approximate best (the approximation errs by ~2^-20).  Each
+        // warpgroup re-scores such groups of its own quarter with exact fp32 squared distances
+        // (lower distance, then lower index, as the oracle); warpgroup 0 merges the quarters.
+        {
           float bv = INFINITY;
 #pragma unroll
           for (int w = 0; w < 4; ++w) bv = fminf(bv, sRes[((j & 1) * 4 + w) * kRowsL + row].x);
           const float lim = bv + kTie;
+          float z[4];  // the block, from the combined rotation in tensor memory
+          {
+            uint32_t zw[4];
+            ptx::tc_fence_after();
+            ptx::tmem_ld4(tmem + lane_base + 4 * j, zw);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int a = 0; a < 4; ++a) z[a] = __uint_as_float(zw[a]);
+          }
           float ev = INFINITY;
           int idx = 0;
-          const float4* cb4 = reinterpret_cast<const float4*>(p.cb);
-          auto resolve = [&](int n0) {  // direct squared distances, as the oracle
-#pragma unroll 8
-            for (int q = 0; q < kPer; ++q) {
+          const float4* cb4 = reinterpret_cast<const float4*>(p.cb) + kPer * wg;
+          auto resolve = [&](int grp, bool take) {  // direct squared distances, as the oracle
+            const int n0 = (grp >> 2) * kChunk + 8 * (grp & 3);  // within this quarter
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
               const float4 c = __ldg(cb4 + n0 + q);
-              const float d0 = zc[0] - c.x, d1 = zc[1] - c.y, d2 = zc[2] - c.z, d3 = zc[3] - c.w;
+              const float d0 = z[0] - c.x, d1 = z[1] - c.y, d2 = z[2] - c.z, d3 = z[3] - c.w;
               const float dd = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
-              if (better(dd, n0 + q, ev, idx)) {
+              const int n = n0 + kPer * wg + q;
+              if (take && better(dd, n, ev, idx)) {
                 ev = dd;
-                idx = n0 + q;
+                idx = n;
               }
             }
           };
-          if (nu > 0.f) {
-#pragma unroll 1
-            for (int w = 0; w < 4; ++w) {
-              const float4 e = sRes[((j & 1) * 4 + w) * kRowsL + row];
-              if (e.x <= lim) resolve(__float_as_int(e.y) * kChunk + kPer * w);
-              const int c2 = __float_as_int(e.w);
-              if (c2 >= 0 && e.z <= lim) resolve(c2 * kChunk + kPer * w);
+          const bool n1 = best <= lim, n2 = sg >= 0 && second <= lim;
+          if (__any_sync(0xffffffffu, n1 || n2)) resolve(n1 ? bg : (n2 ? sg : bg), n1 || n2);
+          if (__any_sync(0xffffffffu, n1 && n2)) resolve(sg >= 0 ? sg : 0, n1 && n2);
+          mine->z = ev;
+          mine->w = __int_as_float(idx);
+          ptx::tc_fence_before();
+        }
+        scan_sync_or(false);
+        if (wg == 0) {
+          float ev = INFINITY;
+          int idx = 0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float4 e = sRes[((j & 1) * 4 + w) * kRowsL + row];
+            if (better(e.z, __float_as_int(e.w), ev, idx)) {
+              ev = e.z;
+              idx = __float_as_int(e.w);
             }
           }
+          if (!(nu > 0.f)) idx = 0;
           const uint32_t bit = (uint32_t)(j * B);
           uint32_t* rw = sRec + row * B;  // this row's record words (B words = 32 B bits)
           rw[bit >> 5] |= (uint32_t)idx << (bit & 31);
