@@ -393,64 +393,129 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def e2e(torch, fq, shape, host, states, args, device, world, dist):
-    """Same metric through the public API with host buffers: every step copies the pinned
-    host cache in, encodes, copies the records out, copies records in, decodes, copies the
-    fp16 result out."""
+def e2e(torch, fq, shape, host, states, args, device, world, dist, chunks=8):
+    """Same metric through the public API with host buffers.  Every step copies the pinned host
+    cache in, encodes, copies the records out, copies them back in, decodes and copies the fp16
+    result out, for each rate.  The step runs in row chunks (each entirely K or V) over three
+    CUDA streams (upload, kernels, download) so that uploads, downloads and kernels overlap.  The step's calls are captured once as a CUDA graph and replayed, as in
+    the device-resident measurement; every byte still crosses the host link in every step."""
     n, d = shape.n, shape.d
     half = n // 2
+    per = half // (chunks // 2)
+    assert per * chunks == n, "chunks must split the K and V halves evenly"
     xh = torch.from_numpy(host).pin_memory()
     xd = torch.empty_like(xh, device=device)
-    outs = []
-    for st in states:
-        outs.append((torch.empty((n, st.P), dtype=torch.uint8).pin_memory(),
-                     torch.empty((n,), dtype=torch.int16).pin_memory()))
-    yh = torch.empty((n, d), dtype=torch.float16).pin_memory()
-    yd = torch.empty((n, d), dtype=torch.float16, device=device)
-    h2d = d2h = 0
+    rec_h = [(torch.empty((n, st.P), dtype=torch.uint8).pin_memory(),
+              torch.empty((n,), dtype=torch.int16).pin_memory()) for st in states]
+    yh = [torch.empty((n, d), dtype=torch.float16).pin_memory() for _ in states]
+    yd = [torch.empty((n, d), dtype=torch.float16, device=device) for _ in states]
+    cs, su, sc, sd = (torch.cuda.Stream(device) for _ in range(4))
+
+    def rows(j):
+        return slice(j * per, (j + 1) * per), ("K" if j < chunks // 2 else "V")
+
+    def mark(stream):
+        e = torch.cuda.Event()
+        e.record(stream)
+        return e
 
     def step():
-        nonlocal h2d, d2h
-        h2d = d2h = 0
-        xd.copy_(xh, non_blocking=True)
-        h2d += xh.numel() * xh.element_size()
-        for st, (ch, nh) in zip(states, outs):
-            cd, nd = st.codes[0], st.norms[0]
-            for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
-                fq.fq_encode(xd[sl], st.rot[t], st.cb, st.rate.k, st.rate.N, codes=cd[sl],
-                             norms=nd[sl], search_index=st.index)
-            ch.copy_(cd, non_blocking=True)
-            nh.copy_(nd, non_blocking=True)
-            d2h += ch.numel() + nh.numel() * 2
-            cd2, nd2 = st.codes[1], st.norms[1]
-            cd2.copy_(ch, non_blocking=True)
-            nd2.copy_(nh, non_blocking=True)
-            h2d += ch.numel() + nh.numel() * 2
-            for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
-                fq.fq_decode(cd2[sl], nd2[sl], st.rot[t], st.cb, d, st.rate.k, st.rate.N, y=yd[sl])
-            yh.copy_(yd, non_blocking=True)
-            d2h += yh.numel() * 2
+        # Enqueued from cs (fork and join).  One stream per copy direction, each in data-flow
+        # order with a lag of one chunk, so that no copy waits behind a later chunk's copies:
+        #   su (upload):   x0 x1 r0 x2 r1 ...    (r = records back in)
+        #   sc (kernels):  e0 e1 d0 e2 d1 ...    (e = encode, d = decode; both rates)
+        #   sd (download): o0 o1 y0 o2 y1 ...    (o = records out, y = fp16 result)
+        e0 = mark(cs)
+        for s_ in (su, sc, sd):
+            s_.wait_event(e0)
+        ev_x, ev_enc, ev_out, ev_in, ev_dec = {}, {}, {}, {}, {}
+        for j in range(chunks + 1):
+            if j < chunks:
+                sl, _ = rows(j)
+                with torch.cuda.stream(su):
+                    xd[sl].copy_(xh[sl], non_blocking=True)
+                ev_x[j] = mark(su)
+            if j >= 1:
+                sl, _ = rows(j - 1)
+                su.wait_event(ev_out[j - 1])
+                with torch.cuda.stream(su):
+                    for r, st in enumerate(states):
+                        ch, nh = rec_h[r]
+                        st.codes[1][sl].copy_(ch[sl], non_blocking=True)
+                        st.norms[1][sl].copy_(nh[sl], non_blocking=True)
+                ev_in[j - 1] = mark(su)
+            if j < chunks:
+                sl, t = rows(j)
+                sc.wait_event(ev_x[j])
+                for st in states:
+                    fq.fq_encode(xd[sl], st.rot[t], st.cb, st.rate.k, st.rate.N,
+                                 codes=st.codes[0][sl], norms=st.norms[0][sl],
+                                 search_index=st.index, stream=sc)
+                ev_enc[j] = mark(sc)
+                sd.wait_event(ev_enc[j])
+                with torch.cuda.stream(sd):
+                    for r, st in enumerate(states):
+                        ch, nh = rec_h[r]
+                        ch[sl].copy_(st.codes[0][sl], non_blocking=True)
+                        nh[sl].copy_(st.norms[0][sl], non_blocking=True)
+                ev_out[j] = mark(sd)
+            if j >= 1:
+                sl, t = rows(j - 1)
+                sc.wait_event(ev_in[j - 1])
+                for r, st in enumerate(states):
+                    fq.fq_decode(st.codes[1][sl], st.norms[1][sl], st.rot[t], st.cb, d,
+                                 st.rate.k, st.rate.N, y=yd[r][sl], stream=sc)
+                ev_dec[j - 1] = mark(sc)
+                sd.wait_event(ev_dec[j - 1])
+                with torch.cuda.stream(sd):
+                    for r in range(len(states)):
+                        yh[r][sl].copy_(yd[r][sl], non_blocking=True)
+        for s_ in (su, sc, sd):
+            cs.wait_event(mark(s_))
 
-    for _ in range(max(3, args.warmup // 10)):
+    h2d = xh.numel() * xh.element_size() + sum(n * st.P + 2 * n for st in states)
+    d2h = sum(n * st.P + 2 * n + n * d * 2 for st in states)
+    main = torch.cuda.current_stream()
+    cs.wait_stream(main)
+    step()  # eager once (library set-up), then capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cs):
         step()
+    torch.cuda.synchronize()
+    for _ in range(max(3, args.warmup // 10)):
+        graph.replay()
+    torch.cuda.synchronize()
+    # the overlapped step must deliver exactly what a plain decode of its records gives
+    for r, st in enumerate(states):
+        ref = torch.empty((n, d), dtype=torch.float16, device=device)
+        for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
+            fq.fq_decode(st.codes[1][sl], st.norms[1][sl], st.rot[t], st.cb, d, st.rate.k,
+                         st.rate.N, y=ref[sl])
+        if not torch.equal(ref.cpu(), yh[r]):
+            raise RuntimeError(f"overlapped end-to-end step disagrees with a plain decode "
+                               f"({st.rate.label})")
     torch.cuda.synchronize()
     reps = max(5, min(50, args.steps // 20))
     if dist is not None:
         dist.barrier()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record()
+    s0.record(main)
     for _ in range(reps):
-        step()
-    s1.record()
+        graph.replay()
+    s1.record(main)
     torch.cuda.synchronize()
     ms = s0.elapsed_time(s1)
+    del graph
     if dist is not None:
         t = torch.tensor([ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     eq = 2 * n * 2 * d * len(states)
     return {"value": round(world * eq * reps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": reps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": reps,
+            "overlap": f"{chunks} row chunks over three CUDA streams (upload, kernels, download) "
+                       "in data-flow order, one CUDA graph per step"}
 
 
 def cpu_baseline(w, args, budget_s: float = 12.0):
