@@ -44,6 +44,16 @@ WORKLOADS = {"gpt2": wl.GPT2, "tinyllama": wl.TINYLLAMA, "large": wl.LARGE, "toy
 
 # ----------------------------------------------------------------------------- helpers
 
+def pick_workload(args):
+    """The named workload; --tokens shrinks its sequences (small cases for profiling only: the
+    bench line then names the reduced workload)."""
+    w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = dataclasses.replace(w, name=f"{w.name}_tokens{args.tokens}",
+                                cache=dataclasses.replace(w.cache, tokens=args.tokens))
+    return w
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -52,10 +62,24 @@ def peaks():
     return 6650.0, "fallback"
 
 
-def source_sha() -> str:
+# The sources each timed kernel is built from (its .cu, the headers it includes and the host
+# launcher that picks it): a recorded DRAM traffic figure only applies while these are unchanged.
+KERNEL_SOURCES = {
+    "encode": ["encode_sm100.cu", "codec_sm100.h", "fq_device.cuh", "sm100_ptx.cuh",
+               "fq_internal.h", "fq_api.cu"],
+    "decode": ["decode_sm100.cu", "codec_sm100.h", "fq_device.cuh", "sm100_ptx.cuh",
+               "fq_internal.h", "fq_api.cu"],
+    "attn": ["attn_sm100.cu", "attn.cu", "fq_device.cuh", "sm100_ptx.cuh", "fq_internal.h",
+             "fq_api.cu"],
+}
+
+
+def source_sha(kernel_label: str) -> str:
+    """Hash of the sources of the kernel a bench label names ("encode_k3N64..." -> encode)."""
+    kind = kernel_label.split("_")[0]
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "random_access_kv_fq_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in KERNEL_SOURCES[kind] + ["../../include/fq.h"]:
+        h.update(open(os.path.join(ROOT, "random_access_kv_fq_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -64,7 +88,7 @@ def profiled_traffic(kernel_label: str):
     for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         for line in open(f):
             m = re.match(r"traffic\s+(\S+)\s+bytes_per_launch=(\d+)\s+source_sha=(\w+)", line)
-            if m and m.group(1) == kernel_label and m.group(3) == source_sha():
+            if m and m.group(1) == kernel_label and m.group(3) == source_sha(kernel_label):
                 return int(m.group(2))
     return None
 
@@ -248,7 +272,7 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    w = WORKLOADS[args.workload]
+    w = pick_workload(args)
     shape0 = w.cache
     step_bytes_est = shape0.n * (shape0.d * 2) * 3 * len(w.rates)
     copies = max(2, math.ceil(2 * L2_BYTES / max(step_bytes_est, 1)) + 1)
@@ -550,7 +574,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = pick_workload(args)
     cb = cpu_baseline(w, args, budget_s=max(3.0, min(20.0, 2.0 * args.steps)))
     line = {"impl": "reference", "metric": "KV encode/decode GB/s (fp16-equiv) & % of roofline; "
             "fused attn us/step", "value": cb["value"], "unit": "GB/s",
@@ -574,6 +598,8 @@ def main(argv=None):
     ap.add_argument("--no-attn", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="shrink the workload's sequence length (small profiling cases)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -2,7 +2,8 @@
 // fp32 input.  This is the reference-grade CUDA path: every step of the encoder and decoder
 // of the FibQuant summary (sec. 2.3) runs here in fp32 with straightforward data movement.
 // The sm_100a fast paths (tensor-core rotation, pruned search, staged records) live in
-// codec_sm100.cu and handle the common shapes; this file covers every other shape.
+// encode_sm100.cu, encode_large_sm100.cu, decode_sm100.cu and decode_large_sm100.cu and handle
+// the common shapes; this file covers every other shape.
 #include <cuda_fp16.h>
 
 #include "fq_device.cuh"

@@ -1,4 +1,5 @@
-// sm_100a fast paths of fq_encode / fq_decode (encode_sm100.cu, encode_large_sm100.cu, decode_sm100.cu).
+// sm_100a fast paths of fq_encode / fq_decode (encode_sm100.cu, encode_large_sm100.cu,
+// decode_sm100.cu, decode_large_sm100.cu).
 #pragma once
 
 #include "fq_internal.h"
@@ -19,6 +20,13 @@ bool encode_large_supported(fq_dtype xt, const Shape& s, const void* x, const vo
 cudaError_t launch_encode_large(const void* x, int64_t n, const Shape& s, const float* rot,
                                 const float* cb, uint8_t* codes, uint16_t* norms,
                                 cudaStream_t st);
+
+// d = 128, k = 4, N <= 4096: tensor-core inverse rotation (decode_large_sm100.cu).
+bool decode_large_supported(fq_dtype yt, const Shape& s, const void* codes, const void* norms,
+                            const void* y, const float* cb);
+cudaError_t launch_decode_large(const uint8_t* codes, const uint16_t* norms, int64_t n,
+                                const Shape& s, const float* rot, const float* cb, void* y,
+                                fq_dtype yt, cudaStream_t st);
 
 bool decode_supported(fq_dtype yt, const Shape& s, const void* codes, const void* norms,
                       const void* y);

@@ -95,6 +95,8 @@ fq_status fq_decode(const uint8_t* codes, const uint16_t* norms, int64_t n, int 
       !aligned(y, y_type == FQ_F16 ? 2 : 4))
     return FQ_ERR_ALIGNMENT;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (sm100::decode_large_supported(y_type, s, codes, norms, y, codebook))
+    return from_cuda(sm100::launch_decode_large(codes, norms, n, s, rot, codebook, y, y_type, cs));
   if (sm100::decode_supported(y_type, s, codes, norms, y))
     return from_cuda(sm100::launch_decode(codes, norms, n, s, rot, codebook, y, y_type, cs));
   return from_cuda(launch_decode_generic(codes, norms, n, s, rot, codebook, y, y_type, cs));

@@ -78,10 +78,12 @@ def check_recon(y, gidx, gnorm_bits, rot, cb, d):
 
 
 def check_recon_f16(y16, ref):
-    """fp16 output: round-to-nearest-even of the fp32 result, so within one fp16 rounding
-    (2^-11 relative per element) of the fp64 reference, plus the fp32 error."""
+    """fp16 output: round-to-nearest-even of the fp32 result, so within one fp16 rounding of
+    the fp64 reference (2^-11 relative per element, and at most 2^-25 absolute below 2^-14,
+    half the subnormal spacing), plus the fp32 error."""
     y = np.asarray(y16, dtype=np.float64)
-    tol = 2.0 ** -11 * np.abs(ref) + 1e-5 * np.linalg.norm(ref, axis=1, keepdims=True)
+    tol = (np.maximum(2.0 ** -11 * np.abs(ref), 2.0 ** -25) +
+           1e-5 * np.linalg.norm(ref, axis=1, keepdims=True))
     assert np.all(np.abs(y - ref) <= tol)
 
 

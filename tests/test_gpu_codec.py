@@ -245,4 +245,28 @@ def test_large_codebook_tensor_core_search(N):
     x = wl.gaussian_rows(1000, d, seed=N, sigma=1.0)
     x[7] = 0  # zero vector
     x[8] = x[9]  # duplicate rows
-    run_codec(x, rot, cb, wl.Rate(k, N, "brute"), d)
+    run_codec(x, rot, cb, wl.Rate(k, N, "brute"), d, out16=True)
+
+
+@pytest.mark.parametrize("B", [2, 5, 8, 9, 12])
+def test_large_decode_tensor_core(B):
+    """d = 128, k = 4: the tensor-core decode of arbitrary records (random indices, random
+    fp16 norms, a zero norm, a ragged last tile) against the oracle decoder, fp32 and fp16 out;
+    several tiles per pipeline."""
+    d, k, N = 128, 4, 1 << B
+    rng = np.random.default_rng(100 + B)
+    rot = tables.rotation(d, wl.ROT_SEED_V)
+    u = rng.standard_normal((N, k))
+    cb = (u / np.linalg.norm(u, axis=1, keepdims=True) *
+          rng.uniform(0.0, 1.0, size=(N, 1))).astype(np.float32)
+    n = 3 * 148 * 2 * 128 + 77
+    idx = rng.integers(0, N, size=(n, d // k))
+    codes = fo.pack(idx, N)
+    norms = rng.uniform(0.0, 40.0, size=n).astype(np.float16)
+    norms[5] = 0
+    ct, nt = torch.from_numpy(codes).cuda(), torch.from_numpy(norms.view(np.int16)).cuda()
+    y = fq.fq_decode(ct, nt, _dev(rot), _dev(cb), d, k, N)
+    y16 = fq.fq_decode(ct, nt, _dev(rot), _dev(cb), d, k, N, out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    ref = par.check_recon(par.to_np(y), idx, norms.view(np.int16), rot, cb, d)
+    par.check_recon_f16(par.to_np(y16).astype(np.float64), ref)
