@@ -20,6 +20,14 @@ bool encode_large_supported(fq_dtype xt, const Shape& s, const void* x, const vo
 cudaError_t launch_encode_large(const void* x, int64_t n, const Shape& s, const float* rot,
                                 const float* cb, uint8_t* codes, uint16_t* norms,
                                 cudaStream_t st);
+// d = 128, k = 4, N = 4096 with a grid index (top-c or exact without overflow lists): tensor-core
+// rotation and a candidate search; an index that does not describe the codebook falls back to
+// exact brute force inside the kernel.
+bool encode_grid_supported(fq_dtype xt, const Shape& s, const void* x, const void* codes,
+                           const float* cb, const void* index);
+cudaError_t launch_encode_grid(const void* x, int64_t n, const float* rot, const float* cb,
+                               const void* index, uint8_t* codes, uint16_t* norms,
+                               cudaStream_t st);
 
 // d = 128, k = 4, N <= 4096: tensor-core inverse rotation (decode_large_sm100.cu).
 bool decode_large_supported(fq_dtype yt, const Shape& s, const void* codes, const void* norms,

@@ -75,6 +75,8 @@ fq_status fq_encode(const void* x, fq_dtype x_type, int64_t n, int d, int k, int
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (sm100::encode_large_supported(x_type, s, x, codes, codebook, search_index))
     return from_cuda(sm100::launch_encode_large(x, n, s, rot, codebook, codes, norms, cs));
+  if (sm100::encode_grid_supported(x_type, s, x, codes, codebook, search_index))
+    return from_cuda(sm100::launch_encode_grid(x, n, rot, codebook, search_index, codes, norms, cs));
   if (sm100::encode_supported(x_type, s, x, codes, norms))
     return from_cuda(sm100::launch_encode(x, x_type, n, s, rot, codebook, codes, norms,
                                           search_index, cs));

@@ -201,6 +201,21 @@ def test_index_with_wrong_codebook_falls_back_to_exact_search():
     assert torch.equal(c1, c2) and torch.equal(n1, n2)
 
 
+def test_large_grid_index_for_another_codebook_falls_back_to_brute_force():
+    """d = 128, N = 4096 with an index built for a 2048-codeword codebook: the grid kernel ignores
+    it and searches all 4096 codewords exactly, matching the oracle's brute force."""
+    d, k, N = 128, 4, 4096
+    rot, cb = tables.rotation(d, wl.ROT_SEED_K), tables.codebook(d, k, N)
+    ix = _dev(fq.fq_build_search_index(cb[:2048], d, k, 2048, fq.FQ_INDEX_TOPC, 8, 4))
+    x = wl.gaussian_rows(300, d, 11)
+    x[3] = 0
+    codes, norms = fq.fq_encode(_dev(x), _dev(rot), _dev(cb), k, N, search_index=ix)
+    torch.cuda.synchronize()
+    enc, _ = _oracle_encode(x, rot, cb, wl.Rate(k, N, "brute"))
+    par.check_records_and_indices(par.to_np(codes), enc, N, d // k)
+    par.check_norms(par.to_np(norms), enc)
+
+
 @pytest.mark.parametrize("dp,k,N", [(64, 2, 16), (66, 3, 64), (64, 4, 8), (64, 2, 256)])
 def test_fast_and_generic_paths_meet_parity_on_the_same_rows(dp, k, N):
     """A 16-byte-aligned fp16 input takes the tensor-core kernel; the same rows behind a
