@@ -44,6 +44,26 @@ WORKLOADS = {"gpt2": wl.GPT2, "tinyllama": wl.TINYLLAMA, "large": wl.LARGE, "toy
 
 # ----------------------------------------------------------------------------- helpers
 
+def rank_cache(w, rank: int):
+    """Rank `rank`'s cache: the workload's shape with its own seed (weak scaling: every rank
+    encodes and decodes a different cache of the same size)."""
+    return dataclasses.replace(w.cache, seed=w.cache.seed + 7919 * rank)
+
+
+def max_over_ranks(torch, dist, ms: float, device) -> float:
+    """The slowest rank's time (the job's time); `ms` itself without a process group."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, bytes_per_rank: float, reps: int, ms: float) -> float:
+    """GB/s of the whole job: every rank moved bytes_per_rank per rep, in ms for all reps."""
+    return world * bytes_per_rank * reps / (ms * 1e-3) / 1e9
+
+
 def pick_workload(args):
     """The named workload; --tokens shrinks its sequences (small cases for profiling only: the
     bench line then names the reduced workload)."""
@@ -172,7 +192,7 @@ class RateState:
 
 
 def build_codec_state(torch, fq, w, rank, copies, device):
-    shape = dataclasses.replace(w.cache, seed=w.cache.seed + 7919 * rank)
+    shape = rank_cache(w, rank)
     n, d = shape.n, shape.d
     half = n // 2
     host = wl.cache(shape)
@@ -323,11 +343,7 @@ def run_gpu(args):
             step_graphs[i % copies].replay()
         t_end.record(stream)
         barrier()
-    total_ms = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(torch, dist, t_start.elapsed_time(t_end), device)
     # per-kernel device time: a graph of every launch of one kind over all copies, replayed
     per = {}
     reps = max(5, min(50, args.steps // copies))
@@ -349,7 +365,7 @@ def run_gpu(args):
         per[lab] = {"ms": ms, "per_step": per_step, "alg_bytes": ab, "kind": kind}
         del g
     step_eq = sum(eb for _, _, _, eb in meta)
-    value = world * step_eq * args.steps / (total_ms * 1e-3) / 1e9
+    value = whole_job_rate(world, step_eq, args.steps, total_ms)
     hbm, hbm_src = peaks()
     dom_lab = max(per, key=lambda k: per[k]["ms"] * per[k]["per_step"])
     dom = per[dom_lab]
@@ -396,7 +412,7 @@ def run_gpu(args):
             agraphs[i % 4].replay()
         a1.record(stream)
         barrier()
-        us = a0.elapsed_time(a1) * 1e3 / areps
+        us = max_over_ranks(torch, dist, a0.elapsed_time(a1), device) * 1e3 / areps
         result["attn"] = {"workload": wl.ATTN.name, "us_per_step": round(us, 2),
                           "bytes_per_step": attn_bytes,
                           "roofline": {"bound": "hbm", "achieved": round(attn_bytes / (us * 1e-6) / 1e9, 1),
@@ -529,14 +545,10 @@ def e2e(torch, fq, shape, host, states, args, device, world, dist, chunks=8):
         graph.replay()
     s1.record(main)
     torch.cuda.synchronize()
-    ms = s0.elapsed_time(s1)
+    ms = max_over_ranks(torch, dist, s0.elapsed_time(s1), device)
     del graph
-    if dist is not None:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
     eq = 2 * n * 2 * d * len(states)
-    return {"value": round(world * eq * reps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    return {"value": round(whole_job_rate(world, eq, reps, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": reps,
             "overlap": f"{chunks} row chunks over three CUDA streams (upload, kernels, download) "
                        "in data-flow order, one CUDA graph per step"}
