@@ -647,3 +647,105 @@ def encode_grid_topc(x: np.ndarray, rot: np.ndarray, codebook: np.ndarray, k: in
     bd = (np.abs(t - nearest_face) * h).min(axis=2)
     norms = nu.astype(np.float16)
     return Encoded(idx, norms, gap, z, nu), bd
+
+
+# --------------------------------------------------------------------------------------
+# Variants (not on the measured path yet).
+#
+# [BQ] key design 3, target-aware scalar rescale: after the inverse rotation the unscaled
+# reconstruction xbar = Pi^T zbar of a unit vector has a shrunk norm.  With the alignment
+# rho = <z, zbar> (= <x, xbar> for unit x) the decoder scales xbar by
+#   S = rho / |xbar|^2   (least squared reconstruction error),
+#   S = 1 / rho          (inner products unbiased: the component along x becomes exact),
+#   S = 1                (plain reconstruction, the rule of the measured path).
+# rho is one more stored scalar per vector.  Readings: |xbar| = |zbar| (Pi is orthogonal, and
+# the padded coordinates are kept before the final truncation to d); a zero vector stores
+# rho = 1.
+# --------------------------------------------------------------------------------------
+
+RESCALE_RULES = ("mse", "unbiased", "plain")
+
+
+def rescale_factor(rho: np.ndarray, zbar_sq: np.ndarray, rule: str) -> np.ndarray:
+    """S of [BQ] key design 3 for alignment rho and squared reconstruction norm |zbar|^2."""
+    rho = np.asarray(rho, dtype=np.float64)
+    if rule == "mse":
+        return rho / np.asarray(zbar_sq, dtype=np.float64)
+    if rule == "unbiased":
+        return 1.0 / rho
+    if rule == "plain":
+        return np.ones_like(rho)
+    raise ValueError(rule)
+
+
+def encode_rescaled(x: np.ndarray, rot: np.ndarray, codebook: np.ndarray, k: int):
+    """The encoder plus rho = <z, zbar> per vector.  Returns (Encoded, rho)."""
+    enc = encode(x, rot, codebook, k)
+    C = np.asarray(codebook, dtype=np.float64)
+    n, dp = enc.z.shape
+    zbar = C[enc.idx].reshape(n, dp)
+    rho = np.sum(enc.z * zbar, axis=1)
+    rho[enc.nu == 0] = 1.0
+    return enc, rho
+
+
+def decode_rescaled(idx: np.ndarray, norms_f16: np.ndarray, rho: np.ndarray, rot: np.ndarray,
+                    codebook: np.ndarray, d: int, rule: str) -> np.ndarray:
+    """x_hat = nu * S * (Pi^T zbar)[0:d] with S from `rule` ([BQ] key design 3)."""
+    C = np.asarray(codebook, dtype=np.float64)
+    n, m = idx.shape
+    zbar = C[idx].reshape(n, m * C.shape[1])
+    S = rescale_factor(rho, np.sum(zbar * zbar, axis=1), rule)
+    xr = zbar @ np.asarray(rot, dtype=np.float64)
+    nu = np.asarray(norms_f16, dtype=np.float16).astype(np.float64)
+    return (nu * S)[:, None] * xr[:, :d]
+
+
+# --------------------------------------------------------------------------------------
+# [TQ] sec. 2.2 (QJL, a 1-bit inner-product quantizer): for x in R^d,
+#   Q_qjl(x) = sign(S x),  Q_qjl^{-1}(q) = sqrt(pi/2) / d * S^T q,
+# with S a d x d matrix of iid N(0, 1) entries (drawn here from a seeded PCG64 generator and
+# passed in).  Reading: sign(0) = +1.
+# [TQ] sec. 3.1 (TurboQuant_mse): y = Pi x, each coordinate of y to its nearest centroid of the
+# scalar Lloyd-Max codebook c1 of the coordinate law; dequantize Pi^T c1[idx].
+# [TQ] sec. 3.2 (TurboQuant_prod, inner-product optimal, b bits): Q_mse at b - 1 bits, then
+# Q_qjl of the residual r = x - Q_mse^{-1}(Q_mse(x)) and gamma = |r|_2; the estimate is
+#   Q_mse^{-1}(Q_mse(x)) + gamma * Q_qjl^{-1}(Q_qjl(r)).
+# All vectors are rows; x is on the unit sphere (the norm is stored separately, as above).
+# --------------------------------------------------------------------------------------
+
+def qjl_matrix(d: int, seed: int) -> np.ndarray:
+    return np.random.default_rng(seed).standard_normal((d, d))
+
+
+def qjl_quantize(x: np.ndarray, S: np.ndarray) -> np.ndarray:
+    s = np.atleast_2d(np.asarray(x, dtype=np.float64)) @ S.T   # rows of (S x)^T
+    return np.where(s >= 0.0, 1.0, -1.0)
+
+
+def qjl_dequantize(q: np.ndarray, S: np.ndarray) -> np.ndarray:
+    d = S.shape[0]
+    return math.sqrt(math.pi / 2.0) / d * (np.atleast_2d(q) @ S)  # rows of (S^T q)^T
+
+
+def turboquant_mse_quantize(x: np.ndarray, rot: np.ndarray, c1: np.ndarray) -> np.ndarray:
+    y = np.atleast_2d(np.asarray(x, dtype=np.float64)) @ np.asarray(rot, dtype=np.float64).T
+    return np.argmin(np.abs(y[:, :, None] - np.asarray(c1)[None, None, :]), axis=2)
+
+
+def turboquant_mse_dequantize(idx: np.ndarray, rot: np.ndarray, c1: np.ndarray) -> np.ndarray:
+    return np.asarray(c1, dtype=np.float64)[idx] @ np.asarray(rot, dtype=np.float64)
+
+
+def turboquant_prod_quantize(x: np.ndarray, rot: np.ndarray, c1: np.ndarray, S: np.ndarray):
+    """(idx of Q_mse at the bits of c1, QJL signs of the residual, gamma = |residual|)."""
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    idx = turboquant_mse_quantize(x, rot, c1)
+    r = x - turboquant_mse_dequantize(idx, rot, c1)
+    return idx, qjl_quantize(r, S), np.linalg.norm(r, axis=1)
+
+
+def turboquant_prod_dequantize(idx: np.ndarray, q: np.ndarray, gamma: np.ndarray,
+                               rot: np.ndarray, c1: np.ndarray, S: np.ndarray) -> np.ndarray:
+    return (turboquant_mse_dequantize(idx, rot, c1) +
+            np.asarray(gamma, dtype=np.float64)[:, None] * qjl_dequantize(q, S))
