@@ -749,3 +749,58 @@ def turboquant_prod_dequantize(idx: np.ndarray, q: np.ndarray, gamma: np.ndarray
                                rot: np.ndarray, c1: np.ndarray, S: np.ndarray) -> np.ndarray:
     return (turboquant_mse_dequantize(idx, rot, c1) +
             np.asarray(gamma, dtype=np.float64)[:, None] * qjl_dequantize(q, S))
+
+
+# --------------------------------------------------------------------------------------
+# Random access and the decode-step write path (not on the measured path yet).  [FQ] sec. 1:
+# records are fixed-size at fixed addresses, so any token decodes alone (gather-decode of a
+# token list) and a sequence can end at any length (per-sequence context lengths).  A decode
+# step that appends its own token encodes that token's key and value into the next record slot
+# of its sequence and attends over the cache including it.  Readings: a length counts tokens
+# from position 0; records past a sequence's length are never read (they may hold anything).
+# --------------------------------------------------------------------------------------
+
+def decode_tokens(codes: np.ndarray, norms_f16: np.ndarray, token_ids, rot: np.ndarray,
+                  codebook: np.ndarray, d: int, k: int, N: int) -> np.ndarray:
+    """Decode only the records at token_ids (any order, repeats allowed) of a [T, P] plane."""
+    ids = np.asarray(token_ids, dtype=np.int64)
+    return decode(np.asarray(codes)[ids], np.asarray(norms_f16)[ids], rot, codebook, d, k, N)
+
+
+def _slice_cache(c: CompressedKV, b: int, length: int) -> CompressedKV:
+    return CompressedKV(c.codes[b:b + 1, :, :length], c.norms[b:b + 1, :, :length], c.rot,
+                        c.codebook, c.k, c.N)
+
+
+def attention_decoded_lengths(q: np.ndarray, Kc: CompressedKV, Vc: CompressedKV, d: int,
+                              scale: float, lengths) -> np.ndarray:
+    """attention_decoded with sequence b limited to its first lengths[b] >= 1 tokens."""
+    q = np.asarray(q, dtype=np.float64)
+    out = np.empty(q.shape)
+    for b, length in enumerate(np.asarray(lengths, dtype=np.int64)):
+        out[b:b + 1] = attention_decoded(q[b:b + 1], _slice_cache(Kc, b, int(length)),
+                                         _slice_cache(Vc, b, int(length)), d, scale)
+    return out
+
+
+def _write_token(c: CompressedKV, x_new: np.ndarray, lengths: np.ndarray) -> CompressedKV:
+    """Encode x_new [B, Hkv, d] and store each row in record slot lengths[b] of its sequence."""
+    Bn, Hkv, d = x_new.shape
+    enc = encode(x_new.reshape(Bn * Hkv, d), c.rot, c.codebook, c.k)
+    rec = pack(enc.idx, c.N).reshape(Bn, Hkv, -1)
+    codes, norms = c.codes.copy(), c.norms.copy()
+    for b in range(Bn):
+        codes[b, :, lengths[b]] = rec[b]
+        norms[b, :, lengths[b]] = enc.norms.reshape(Bn, Hkv)[b]
+    return CompressedKV(codes, norms, c.rot, c.codebook, c.k, c.N)
+
+
+def append_and_attend(q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray, Kc: CompressedKV,
+                      Vc: CompressedKV, d: int, scale: float, lengths):
+    """One decode step with its own token: k_new, v_new [B, Hkv, d] are encoded into slot
+    lengths[b] of each sequence (the caches need room), then the step attends over
+    lengths[b] + 1 tokens.  Returns (out, new key cache, new value cache, new lengths)."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    K2 = _write_token(Kc, np.asarray(k_new), lengths)
+    V2 = _write_token(Vc, np.asarray(v_new), lengths)
+    return attention_decoded_lengths(q, K2, V2, d, scale, lengths + 1), K2, V2, lengths + 1
