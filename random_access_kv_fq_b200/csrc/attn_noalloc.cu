@@ -50,13 +50,22 @@ extern "C" fq_status fq_attn_decode_noalloc(
     const uint16_t* k_norms, int kK, int NK, const float* rotK, const float* cbK,
     const uint8_t* v_codes, const uint16_t* v_norms, int kV, int NV, const float* rotV,
     const float* cbV, float scale, float* out, void* stream) {
+  // The same validation as fq_attn_decode comes first, so that a bad call is refused with its
+  // own status before the scratch array is looked up.
+  fq::AttnArgs a;
+  size_t need = 0;
+  fq_status st = fq::attn_prepare(q, B, Hq, Hkv, T, d, k_codes, k_norms, kK, NK, rotK, cbK,
+                                  v_codes, v_norms, kV, NV, rotV, cbV, scale, out, &a, &need);
+  if (st != FQ_OK) return st;
   // Sizes beyond the fixed scratch are refused before anything is enqueued.
-  const size_t need = fq_attn_workspace_bytes(B, Hq, Hkv, T, d, kV);
   if (need > (size_t)FQ_ATTN_NOALLOC_SCRATCH_BYTES) return FQ_ERR_WORKSPACE;
   void* scratch = nullptr;
-  fq_status st = fq::scratch_on_current_device(&scratch);
-  if (st != FQ_OK) return st;
-  // Same validation, kernels and results as fq_attn_decode, with the fixed array as workspace.
+  if (need > 0) {
+    st = fq::scratch_on_current_device(&scratch);
+    if (st != FQ_OK) return st;
+  }
+  // Same kernels and results as fq_attn_decode, with the fixed array as workspace (T = 0 needs
+  // none: the output is zeroed).
   return fq_attn_decode(q, B, Hq, Hkv, T, d, k_codes, k_norms, kK, NK, rotK, cbK, v_codes,
                         v_norms, kV, NV, rotV, cbV, scale, out, scratch,
                         (size_t)FQ_ATTN_NOALLOC_SCRATCH_BYTES, stream);

@@ -104,6 +104,10 @@ fq_status fq_decode(const uint8_t* codes, const uint16_t* norms, int64_t n, int 
   return from_cuda(launch_decode_generic(codes, norms, n, s, rot, codebook, y, y_type, cs));
 }
 
+}  // extern "C"
+
+namespace fq {
+
 static fq_status attn_shapes(int B, int Hq, int Hkv, int64_t T, int d, int kK, int NK, int kV,
                              int NV, Shape* ks, Shape* vs) {
   if (B < 1 || Hq < 1 || Hkv < 1 || T < 0 || Hq % Hkv != 0) return FQ_ERR_INVALID_ARG;
@@ -115,6 +119,50 @@ static fq_status attn_shapes(int B, int Hq, int Hkv, int64_t T, int d, int kK, i
   if (NK > 1024 || NV > 1024) return FQ_ERR_UNSUPPORTED;
   return FQ_OK;
 }
+
+fq_status attn_prepare(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int d,
+                       const uint8_t* k_codes, const uint16_t* k_norms, int kK, int NK,
+                       const float* rotK, const float* cbK, const uint8_t* v_codes,
+                       const uint16_t* v_norms, int kV, int NV, const float* rotV,
+                       const float* cbV, float scale, float* out, AttnArgs* a, size_t* need) {
+  *need = 0;
+  fq_status st = attn_shapes(B, Hq, Hkv, T, d, kK, NK, kV, NV, &a->ks, &a->vs);
+  if (st != FQ_OK) return st;
+  if (!std::isfinite(scale)) return FQ_ERR_INVALID_ARG;
+  if (!q || !out) return FQ_ERR_INVALID_ARG;
+  if (T == 0) return FQ_OK;
+  if (!k_codes || !k_norms || !rotK || !cbK || !v_codes || !v_norms || !rotV || !cbV)
+    return FQ_ERR_INVALID_ARG;
+  if (!aligned(q, 2) || !aligned(k_norms, 2) || !aligned(v_norms, 2) || !aligned(rotK, 4) ||
+      !aligned(cbK, 4) || !aligned(rotV, 4) || !aligned(cbV, 4) || !aligned(out, 4))
+    return FQ_ERR_ALIGNMENT;
+  a->q = q;
+  a->B = B;
+  a->Hq = Hq;
+  a->Hkv = Hkv;
+  a->T = T;
+  a->d = d;
+  a->k_codes = k_codes;
+  a->k_norms = k_norms;
+  a->rotK = rotK;
+  a->cbK = cbK;
+  a->v_codes = v_codes;
+  a->v_norms = v_norms;
+  a->rotV = rotV;
+  a->cbV = cbV;
+  a->scale = scale;
+  a->out = out;
+  a->partials = nullptr;
+  a->splits = attn_splits(B, Hkv, T);
+  a->tokens_per_split = attn_tokens_per_split(T, a->splits);
+  *need = attn_partials_bytes(B, Hq, a->splits, a->vs.dp);
+  if (attn_smem_bytes(*a) > 200 * 1024) return FQ_ERR_UNSUPPORTED;
+  return FQ_OK;
+}
+
+}  // namespace fq
+
+extern "C" {
 
 size_t fq_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int d, int kV) {
   Shape ks, vs;
@@ -131,41 +179,16 @@ fq_status fq_attn_decode(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, i
                          const float* cbV, float scale, float* out, void* workspace,
                          size_t workspace_bytes, void* stream) {
   AttnArgs a;
-  fq_status st = attn_shapes(B, Hq, Hkv, T, d, kK, NK, kV, NV, &a.ks, &a.vs);
+  size_t need = 0;
+  fq_status st = attn_prepare(q, B, Hq, Hkv, T, d, k_codes, k_norms, kK, NK, rotK, cbK, v_codes,
+                              v_norms, kV, NV, rotV, cbV, scale, out, &a, &need);
   if (st != FQ_OK) return st;
-  if (!std::isfinite(scale)) return FQ_ERR_INVALID_ARG;
-  if (!q || !out) return FQ_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (T == 0)
     return from_cuda(cudaMemsetAsync(out, 0, (size_t)B * Hq * d * sizeof(float), cs));
-  if (!k_codes || !k_norms || !rotK || !cbK || !v_codes || !v_norms || !rotV || !cbV)
-    return FQ_ERR_INVALID_ARG;
-  if (!aligned(q, 2) || !aligned(k_norms, 2) || !aligned(v_norms, 2) || !aligned(rotK, 4) ||
-      !aligned(cbK, 4) || !aligned(rotV, 4) || !aligned(cbV, 4) || !aligned(out, 4))
-    return FQ_ERR_ALIGNMENT;
-  a.q = q;
-  a.B = B;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.T = T;
-  a.d = d;
-  a.k_codes = k_codes;
-  a.k_norms = k_norms;
-  a.rotK = rotK;
-  a.cbK = cbK;
-  a.v_codes = v_codes;
-  a.v_norms = v_norms;
-  a.rotV = rotV;
-  a.cbV = cbV;
-  a.scale = scale;
-  a.out = out;
-  a.splits = attn_splits(B, Hkv, T);
-  a.tokens_per_split = attn_tokens_per_split(T, a.splits);
-  size_t need = attn_partials_bytes(B, Hq, a.splits, a.vs.dp);
   if (!workspace || workspace_bytes < need) return FQ_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return FQ_ERR_ALIGNMENT;
   a.partials = static_cast<float*>(workspace);
-  if (attn_smem_bytes(a) > 200 * 1024) return FQ_ERR_UNSUPPORTED;
   return from_cuda(launch_attn(a, cs));
 }
 

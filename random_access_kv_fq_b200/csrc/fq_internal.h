@@ -97,6 +97,13 @@ struct AttnArgs {
   int splits;
   int64_t tokens_per_split;
 };
+// Validates the arguments of fq_attn_decode (everything but the workspace) and fills `a` and
+// the workspace bytes the call needs; nothing is enqueued.  T = 0 returns FQ_OK with *need = 0.
+fq_status attn_prepare(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int d,
+                       const uint8_t* k_codes, const uint16_t* k_norms, int kK, int NK,
+                       const float* rotK, const float* cbK, const uint8_t* v_codes,
+                       const uint16_t* v_norms, int kV, int NV, const float* rotV,
+                       const float* cbV, float scale, float* out, AttnArgs* a, size_t* need);
 int attn_splits(int B, int Hkv, int64_t T);
 int64_t attn_tokens_per_split(int64_t T, int splits);
 size_t attn_partials_bytes(int B, int Hq, int splits, int dpV);

@@ -52,8 +52,6 @@ def test_attention_small(T):
     q, Kc, Vc, _, _ = _setup(w)
     scale = 1 / math.sqrt(w.d)
     ref = fo.attention_decoded(q, Kc, Vc, w.d, scale)
-    lut = fo.attention_lut(q, Kc, Vc, w.d, scale)
-    np.testing.assert_allclose(lut, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
     out = _gpu_attn(q, Kc, Vc, scale)
     par.check_attention(out, ref)
 

@@ -99,6 +99,35 @@ def test_entry_points_validate_before_touching_the_device():
     assert fq.fq_attn_workspace_bytes(1, 3, 2, 10, 64, 3) == 0
 
 
+def test_noalloc_attention_validates_like_the_workspace_entry_point():
+    """The allocation-free attention entry point refuses a bad call with the same status as
+    fq_attn_decode, on the host, before it looks up its scratch array (no CUDA call is made, so
+    this runs without a GPU)."""
+    L = _lib.lib()
+    base = [16, 1, 32, 4, 100, 64, 16, 16, 2, 16, 16, 16, 16, 16, 3, 64, 16, 16,
+            ctypes.c_float(0.125), 16, None]
+    bad = {
+        "Hq not a multiple of Hkv": ({2: 6}, 1),
+        "group too large": ({2: 34, 3: 2}, 2),
+        "d above 128": ({5: 200}, 2),
+        "N not a power of two": ({9: 15}, 2),
+        "non-finite scale": ({18: ctypes.c_float(float("nan"))}, 1),
+        "null query": ({0: None}, 1),
+        "null key records": ({6: None}, 1),
+        "misaligned norms": ({7: 17}, 3),
+        "scratch too small": ({1: 64, 2: 256, 3: 16, 4: 1024}, 4),
+    }
+    for why, (edits, status) in bad.items():
+        ws_args = list(base[:20]) + [None, 0, None]
+        na_args = list(base)
+        for i, v in edits.items():
+            na_args[i] = v
+            ws_args[i] = v
+        assert L.fq_attn_decode_noalloc(*na_args) == status, why
+        if status != 4:
+            assert L.fq_attn_decode(*ws_args) == status, why
+
+
 # ---------------------------------------------------------------- host index builder
 
 def _cell_of(z, hdr):
