@@ -54,7 +54,7 @@ typedef enum {
   FQ_ERR_ALIGNMENT = 3,   /* a pointer that breaks a stated alignment rule */
   FQ_ERR_WORKSPACE = 4,   /* workspace / index buffer missing or too small */
   FQ_ERR_CUDA = 5,        /* a CUDA launch or runtime call failed */
-  FQ_ERR_TIMEOUT = 6      /* reserved: a bounded device-side wait gave up */
+  FQ_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (see fq_wait_status) */
 } fq_status;
 
 typedef enum { FQ_F16 = 0, FQ_F32 = 1 } fq_dtype;
@@ -161,6 +161,32 @@ fq_status fq_attn_decode_noalloc(const uint16_t* q, int B, int Hq, int Hkv, int6
                                  const uint8_t* v_codes, const uint16_t* v_norms, int kV,
                                  int NV, const float* rotV, const float* cbV, float scale,
                                  float* out, void* stream);
+
+/*
+ * fq_wait_status - reports kernels whose bounded device-side waits gave up.
+ *
+ * Every wait inside the library's kernels (for an asynchronous copy, a tensor-core operation or
+ * another warp's hand-off) gives up after a bounded number of polls instead of hanging the GPU.
+ * A CTA whose wait gave up stops its loop, lets its own copies and tensor-core work in flight
+ * land, frees its tensor memory, adds one to a per-GPU failure count and exits; the outputs of
+ * that launch are then unspecified.  Launches are asynchronous, so the entry points above cannot
+ * return FQ_ERR_TIMEOUT themselves; this call reports it.
+ *   timed_out  (host, out, may be NULL) the number of CTAs whose waits gave up on the current
+ *              device since the count was last cleared.
+ *   clear      nonzero: reset the count to zero after reading it.
+ * Waits for all work on the current device first (cudaDeviceSynchronize), so do not call it
+ * inside a stream capture.  Returns FQ_ERR_TIMEOUT when the count is nonzero, FQ_OK when it is
+ * zero, FQ_ERR_CUDA when the device cannot be queried.
+ */
+fq_status fq_wait_status(unsigned* timed_out, int clear);
+
+/*
+ * fq_selftest_wait_timeout - diagnostic for the failure path (no counterpart in the paper).
+ * Enqueues on `stream` one small kernel whose single wait is on an mbarrier phase that nothing
+ * ever completes; it polls `polls` times (1 .. 2^20), gives up exactly as the codec kernels do
+ * and counts one timed-out wait, which fq_wait_status then reports.  Nothing faults or hangs.
+ */
+fq_status fq_selftest_wait_timeout(uint32_t polls, void* stream);
 
 /*
  * fq_build_search_index - builds, on the HOST, the candidate table fq_encode can use instead

@@ -8,4 +8,5 @@ not load the library; the first compute call does, and raises if it is missing.
 from ._lib import (FQ_ATTN_NOALLOC_SCRATCH_BYTES, FQ_F16, FQ_F32, FQ_INDEX_EXACT,  # noqa: F401
                    FQ_INDEX_TOPC, FQError,
                    fq_attn_decode, fq_attn_decode_noalloc, fq_attn_workspace_bytes, fq_build_search_index, fq_decode,
-                   fq_encode, fq_padded_dim, fq_payload_bytes, lib, status_string)
+                   fq_encode, fq_padded_dim, fq_payload_bytes, fq_wait_status, lib,
+                   status_string)

@@ -41,6 +41,8 @@ _SIGS = {
                             ctypes.c_float, _vp, _vp, _sz, _vp]),
     "fq_build_search_index": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _sz,
                                    ctypes.POINTER(_sz)]),
+    "fq_wait_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i]),
+    "fq_selftest_wait_timeout": (_i, [ctypes.c_uint32, _vp]),
     "fq_attn_decode_noalloc": (_i, [_vp, _i, _i, _i, _c_i64, _i,
                                     _vp, _vp, _i, _i, _vp, _vp,
                                     _vp, _vp, _i, _i, _vp, _vp,
@@ -195,6 +197,16 @@ def fq_attn_decode_noalloc(q, k_codes, k_norms, kK: int, NK: int, rotK, cbK, v_c
                                       float(scale), _ptr(out), _stream(stream))
     _check("fq_attn_decode_noalloc", st)
     return out
+
+
+def fq_wait_status(clear: bool = False) -> int:
+    """Number of CTAs whose bounded device-side waits gave up on the current device (waits for
+    the device first).  0 means no launch since the last clear lost a wait."""
+    n = ctypes.c_uint(0)
+    st = lib().fq_wait_status(ctypes.byref(n), 1 if clear else 0)
+    if st not in (0, 6):
+        _check("fq_wait_status", st)
+    return int(n.value)
 
 
 def fq_build_search_index(codebook, d: int, k: int, N: int, kind: int, L: int,

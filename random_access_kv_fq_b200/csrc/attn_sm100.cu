@@ -744,4 +744,8 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t st) {
 }
 
 }  // namespace attn100
+cudaError_t wait_timeouts_attn(bool clear, unsigned* count) {
+  return read_wait_counter(g_fq_wait_timeouts, clear, count);
+}
+
 }  // namespace fq

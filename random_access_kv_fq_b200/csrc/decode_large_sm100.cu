@@ -345,4 +345,8 @@ cudaError_t launch_decode_large(const uint8_t* codes, const uint16_t* norms, int
 }
 
 }  // namespace sm100
+cudaError_t wait_timeouts_decode_large(bool clear, unsigned* count) {
+  return read_wait_counter(sm100::g_decl_wait_timeouts, clear, count);
+}
+
 }  // namespace fq

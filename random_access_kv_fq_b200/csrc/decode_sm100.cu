@@ -624,4 +624,8 @@ cudaError_t launch_decode(const uint8_t* codes, const uint16_t* norms, int64_t n
 }
 
 }  // namespace sm100
+cudaError_t wait_timeouts_decode(bool clear, unsigned* count) {
+  return read_wait_counter(sm100::g_dec_wait_timeouts, clear, count);
+}
+
 }  // namespace fq

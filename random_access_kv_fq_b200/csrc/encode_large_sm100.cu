@@ -859,4 +859,8 @@ cudaError_t launch_encode_large(const void* x, int64_t n, const Shape& s, const 
 }
 
 }  // namespace sm100
+cudaError_t wait_timeouts_encode_large(bool clear, unsigned* count) {
+  return read_wait_counter(sm100::g_encl_wait_timeouts, clear, count);
+}
+
 }  // namespace fq

@@ -678,4 +678,8 @@ cudaError_t launch_encode(const void* x, fq_dtype, int64_t n, const Shape& s, co
 }
 
 }  // namespace sm100
+cudaError_t wait_timeouts_encode(bool clear, unsigned* count) {
+  return read_wait_counter(sm100::g_enc_wait_timeouts, clear, count);
+}
+
 }  // namespace fq

@@ -192,4 +192,21 @@ fq_status fq_attn_decode(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, i
   return from_cuda(launch_attn(a, cs));
 }
 
+fq_status fq_wait_status(unsigned* timed_out, int clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FQ_ERR_CUDA;
+  unsigned n = 0;
+  cudaError_t (*readers[])(bool, unsigned*) = {wait_timeouts_encode, wait_timeouts_encode_large,
+                                               wait_timeouts_decode, wait_timeouts_decode_large,
+                                               wait_timeouts_attn, wait_timeouts_selftest};
+  for (auto rd : readers)
+    if (rd(clear != 0, &n) != cudaSuccess) return FQ_ERR_CUDA;
+  if (timed_out) *timed_out = n;
+  return n ? FQ_ERR_TIMEOUT : FQ_OK;
+}
+
+fq_status fq_selftest_wait_timeout(uint32_t polls, void* stream) {
+  if (polls < 1 || polls > (1u << 20)) return FQ_ERR_INVALID_ARG;
+  return from_cuda(launch_selftest_wait(polls, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -111,6 +111,30 @@ size_t attn_smem_bytes(const AttnArgs& a);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t st);
 
+// ---- bounded-wait failure counters ---------------------------------------------------------
+// Every kernel file whose kernels wait on mbarriers keeps a __device__ count of the CTAs whose
+// bounded waits gave up.  Its reader adds that count on the current device to *count and zeroes
+// it when `clear` is set (synchronous copies; the caller synchronises the device first).
+template <class Sym>
+inline cudaError_t read_wait_counter(const Sym& sym, bool clear, unsigned* count) {
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, sym, sizeof(v));
+  if (e != cudaSuccess) return e;
+  *count += v;
+  if (clear && v != 0) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(sym, &zero, sizeof(zero));
+  }
+  return e;
+}
+cudaError_t wait_timeouts_encode(bool clear, unsigned* count);        // encode_sm100.cu
+cudaError_t wait_timeouts_encode_large(bool clear, unsigned* count);  // encode_large_sm100.cu
+cudaError_t wait_timeouts_decode(bool clear, unsigned* count);        // decode_sm100.cu
+cudaError_t wait_timeouts_decode_large(bool clear, unsigned* count);  // decode_large_sm100.cu
+cudaError_t wait_timeouts_attn(bool clear, unsigned* count);          // attn_sm100.cu
+cudaError_t wait_timeouts_selftest(bool clear, unsigned* count);      // selftest.cu
+cudaError_t launch_selftest_wait(uint32_t polls, cudaStream_t st);     // selftest.cu
+
 // sm_100a tensor-core attention (attn_sm100.cu) for the shapes it supports.
 namespace attn100 {
 bool supported(const AttnArgs& a);

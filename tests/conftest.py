@@ -32,3 +32,15 @@ def cuda_device():
     import torch
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     return torch.device("cuda:0")
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _no_bounded_wait_gave_up(request):
+    """After every GPU test module: no kernel of the library gave up a bounded wait (a timed-out
+    wait leaves unspecified outputs, so parity alone could miss it)."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import random_access_kv_fq_b200 as fq
+    n = fq.fq_wait_status(clear=True)
+    assert n == 0, f"{n} CTAs gave up a bounded wait during {request.node.name}"
