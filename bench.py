@@ -1,16 +1,23 @@
 """Benchmark of the FibQuant KV codec hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fibquant|reference]
-                    [--workload gpt2|tinyllama|large|toy]
+                    [--workload large|gpt2|tinyllama|toy] [--tokens T]
+                    [--no-configs] [--no-attn] [--no-e2e] [--no-cpu]
 
-One step = one pass of the whole hot path over the workload's synthetic GPT-2-small-shaped
-KV cache (12 layers x 12 heads x 1024 tokens, K and V, d = 64, fp16): for each of its two
-rates (k=3 N=64 with the exact grid search, k=4 N=8 with brute force) encode K and V
-(separate rotations) and decode K and V to fp16.  The metric is fp16-equivalent GB/s:
-(encode input + decode output) bytes as an fp16 cache, divided by the step time.  The fused
-decode-attention step (B16, Hq32/Hkv4, T32768, d64) is timed in the same run and reported
-under "attn".  Inputs rotate over enough copies that every kernel reads data that has left
-the 126 MB L2 (the whole-step footprint between reuses is >= 2x L2).
+Headline (the line's "value"): the large-codebook KV cache, 32 layers x 8 kv heads x 32768
+tokens, d = 128, K and V (16,777,216 vectors, 4.3 GB of fp16), at k = 4, N = 4096 with the top-8
+grid search (L = 16 cells per axis).  One step encodes K and V (separate rotations) and decodes
+both back to fp16; the metric is fp16-equivalent GB/s: (encode input + decode output) bytes as an
+fp16 cache, divided by the step time.  The same cache's exact brute-force encode (tensor-core
+distance contraction with fp32 re-ranking) is timed as a second labelled kernel under
+"extra_kernels".  In the same run: the GPT-2-small-shaped, TinyLlama-shaped and toy caches under
+"configs" (their own steps: every rate, encode + decode of K and V), the fused decode-attention
+step (B16, Hq32/Hkv4, T32768, d64) under "attn", the end-to-end figure through the C ABI with
+host buffers under "e2e", and the CPU oracle on the host's cores under "cpu_baseline".
+
+Inputs larger than 2x the 126 MB L2 stream from HBM; the smaller caches rotate over enough
+copies that every kernel reads data that has left L2.  Device times are CUDA events on the
+launching stream, around CUDA-graph replays of the step's C-ABI calls.
 
 With --gpus N > 1 (launched by torch.distributed.run), every rank processes its own cache of
 the same shape (weak scaling, no data-path collective); the time is the max over ranks.
@@ -20,11 +27,9 @@ from __future__ import annotations
 import argparse
 import dataclasses
 import hashlib
-import glob
 import json
 import math
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -39,7 +44,9 @@ sys.path.insert(0, ROOT)
 from random_access_kv_fq_b200 import workloads as wl  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
-WORKLOADS = {"gpt2": wl.GPT2, "tinyllama": wl.TINYLLAMA, "large": wl.LARGE, "toy": wl.TOY}
+WORKLOADS = {"large": wl.LARGE, "gpt2": wl.GPT2, "tinyllama": wl.TINYLLAMA, "toy": wl.TOY}
+METRIC = "KV encode/decode GB/s (fp16-equiv) & % of roofline; fused attn us/step"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -64,14 +71,23 @@ def whole_job_rate(world: int, bytes_per_rank: float, reps: int, ms: float) -> f
     return world * bytes_per_rank * reps / (ms * 1e-3) / 1e9
 
 
-def pick_workload(args):
+def pick_workload(args, key=None):
     """The named workload; --tokens shrinks its sequences (small cases for profiling only: the
     bench line then names the reduced workload)."""
-    w = WORKLOADS[args.workload]
-    if args.tokens:
+    w = WORKLOADS[key or args.workload]
+    if getattr(args, "tokens", None):
         w = dataclasses.replace(w, name=f"{w.name}_tokens{args.tokens}",
                                 cache=dataclasses.replace(w.cache, tokens=args.tokens))
     return w
+
+
+def step_and_extra_rates(w):
+    """(rates in the timed step, rates timed only as extra encode kernels).  For the large
+    codebook the exact brute-force encode is a second labelled kernel, not part of the step."""
+    if w.cache.d == 128:
+        return (tuple(r for r in w.rates if r.search != "brute"),
+                tuple(r for r in w.rates if r.search == "brute"))
+    return tuple(w.rates), ()
 
 
 def peaks():
@@ -82,103 +98,147 @@ def peaks():
     return 6650.0, "fallback"
 
 
-# The sources each timed kernel is built from (its .cu, the headers it includes and the host
-# launcher that picks it): a recorded DRAM traffic figure only applies while these are unchanged.
+# The sources a timed kernel is built from (its .cu files, the headers they include and the host
+# code that picks them): a recorded DRAM traffic figure only applies while these are unchanged.
+_COMMON = ["fq_device.cuh", "sm100_ptx.cuh", "fq_internal.h", "fq_api.cu", "codec_sm100.h"]
 KERNEL_SOURCES = {
-    "encode": ["encode_sm100.cu", "codec_sm100.h", "fq_device.cuh", "sm100_ptx.cuh",
-               "fq_internal.h", "fq_api.cu"],
-    "decode": ["decode_sm100.cu", "codec_sm100.h", "fq_device.cuh", "sm100_ptx.cuh",
-               "fq_internal.h", "fq_api.cu"],
-    "attn": ["attn_sm100.cu", "attn.cu", "fq_device.cuh", "sm100_ptx.cuh", "fq_internal.h",
-             "fq_api.cu"],
+    ("encode", 64): ["encode_sm100.cu", "codec_generic.cu"],
+    ("decode", 64): ["decode_sm100.cu", "codec_generic.cu"],
+    ("encode", 128): ["encode_large_sm100.cu", "codec_generic.cu"],
+    ("decode", 128): ["decode_large_sm100.cu", "codec_generic.cu"],
+    ("attn", 64): ["attn_sm100.cu", "attn.cu"],
 }
 
 
-def source_sha(kernel_label: str) -> str:
+def source_sha(kernel_label: str, d: int = 64) -> str:
     """Hash of the sources of the kernel a bench label names ("encode_k3N64..." -> encode)."""
     kind = kernel_label.split("_")[0]
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES[kind] + ["../../include/fq.h"]:
+    for f in KERNEL_SOURCES[(kind, d)] + _COMMON:
         h.update(open(os.path.join(ROOT, "random_access_kv_fq_b200", "csrc", f), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "fq.h"), "rb").read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_label: str):
-    """Per-launch DRAM bytes recorded from an ncu capture of this exact source, else None."""
-    for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
-        for line in open(f):
-            m = re.match(r"traffic\s+(\S+)\s+bytes_per_launch=(\d+)\s+source_sha=(\w+)", line)
-            if m and m.group(1) == kernel_label and m.group(3) == source_sha(kernel_label):
-                return int(m.group(2))
-    return None
+def traffic_key(workload_name: str, label: str) -> str:
+    base = workload_name.split("_tokens")[0]
+    return f"{base}/{label}"
+
+
+def profiled_traffic(workload_name: str, label: str, d: int, vectors: int):
+    """Per-launch DRAM bytes (read + write) from an ncu capture of this exact source, scaled to
+    `vectors` per launch, else None.  The record under profiles/traffic.json holds the bytes per
+    vector of the captured launch and the source hash it was taken on."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    rec = json.load(open(TRAFFIC_FILE)).get(traffic_key(workload_name, label))
+    if not rec or rec.get("source_sha") != source_sha(label, d):
+        return None
+    return int(round(rec["bytes_per_vector"] * vectors))
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """SM clock and clock-event reasons sampled every 10 ms (NVML) while the timed region runs;
+    falls back to `nvidia-smi -lms 100` when NVML is unavailable."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+            "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, torch, device_index: int, period_s: float = 0.01):
+        self.torch, self.dev, self.period = torch, device_index, period_s
+        self.samples = []   # (time, sm_mhz, max_mhz, reasons bitmask)
+        self.stop = threading.Event()
+        self.thread = None
         self.proc = None
-        self.lines = []   # (arrival time, line)
         self.t0 = self.t1 = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = self.torch.cuda.get_device_properties(self.dev)
+        uuid = str(props.uuid)
+        for u in (uuid, "GPU-" + uuid):
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(u)
+            except Exception:
+                pass
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-            deadline = time.time() + 5.0  # the sampler is running before the region starts
-            while not self.lines and time.time() < deadline and self.proc.poll() is None:
-                time.sleep(0.01)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            nv, h = self._nvml_handle()
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+            def run():
+                while not self.stop.is_set():
+                    try:
+                        self.samples.append((time.time(),
+                                             float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                             mx, int(reasons(h))))
+                    except Exception:
+                        pass
+                    self.stop.wait(self.period)
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+        except Exception:
+            self._smi()
+        deadline = time.time() + 5.0  # the sampler runs before the region starts
+        while not self.samples and time.time() < deadline:
+            time.sleep(0.005)
         self.t0 = time.time()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+    def _smi(self):
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={fields}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+
+        def read():
+            for line in self.proc.stdout:
+                p = [x.strip() for x in line.split(",")]
+                try:
+                    bits = sum(b for (nm, b), v in zip(self.BITS.items(), p[2:6])
+                               if v.lower().startswith("active"))
+                    self.samples.append((time.time(), float(p[0]), float(p[1]), bits))
+                except (ValueError, IndexError):
+                    pass
+        self.thread = threading.Thread(target=read, daemon=True)
+        self.thread.start()
 
     def __exit__(self, *a):
         self.t1 = time.time()
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ts, ln in self.lines:
-            if self.t0 is not None and not (self.t0 <= ts <= self.t1 + 0.1):
-                continue  # only samples taken while the timed region ran
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
+        inside = [s for s in self.samples
+                  if self.t0 is not None and self.t0 <= s[0] <= self.t1 + 0.02]
+        if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = sorted({nm for _, _, _, bits in inside for nm, b in self.BITS.items() if bits & b})
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": inside[-1][2],
+                "reasons": reasons, "samples": len(inside),
+                "source": "nvml 10 ms" if self.proc is None else "nvidia-smi 100 ms"}
 
 
-# ----------------------------------------------------------------------------- workload setup
+# ----------------------------------------------------------------------------- codec state
 
 @dataclasses.dataclass
 class RateState:
@@ -191,16 +251,34 @@ class RateState:
     norms: list      # per copy: [n] int16
 
 
-def build_codec_state(torch, fq, w, rank, copies, device):
+@dataclasses.dataclass
+class CodecRun:
+    w: object
+    shape: object
+    host: object
+    xs: list
+    ys: list
+    step: list       # RateState of the rates in the step
+    extra: list      # RateState of the rates timed only as extra encode kernels
+    copies: int
+
+
+def build_codec_run(torch, fq, w, rank, device, with_extra=True):
+    from random_access_kv_fq_b200 import tables
     shape = rank_cache(w, rank)
     n, d = shape.n, shape.d
     half = n // 2
-    host = wl.cache(shape)
-    tdtype = torch.float16 if shape.dtype == "f16" else torch.float32
+    step_rates, extra_rates = step_and_extra_rates(w)
+    if not with_extra:
+        extra_rates = ()
+    in_bytes = n * d * (2 if shape.dtype == "f16" else 4)
+    # enough input copies that a kernel never finds its input still in L2 (>= 2x L2 between reuses)
+    copies = 1 if in_bytes >= 2 * L2_BYTES else min(8, max(2, math.ceil(2 * L2_BYTES / in_bytes) + 1))
+    host = wl.cache(shape, workers=min(32, len(os.sched_getaffinity(0))))
     xs = [torch.from_numpy(host).to(device) for _ in range(copies)]
-    from random_access_kv_fq_b200 import tables
-    states = []
-    for rate in w.rates:
+    tdtype = torch.float16
+
+    def rate_state(rate, ncopies):
         dp = fq.fq_padded_dim(d, rate.k)
         rot = {"K": torch.from_numpy(tables.rotation(dp, wl.ROT_SEED_K)).to(device),
                "V": torch.from_numpy(tables.rotation(dp, wl.ROT_SEED_V)).to(device)}
@@ -212,38 +290,150 @@ def build_codec_state(torch, fq, w, rank, copies, device):
             index = torch.from_numpy(fq.fq_build_search_index(cb_np, d, rate.k, rate.N, kind,
                                                               rate.grid_L, rate.grid_c)).to(device)
         P = fq.fq_payload_bytes(d, rate.k, rate.N)
-        codes = [torch.empty((n, P), dtype=torch.uint8, device=device) for _ in range(copies)]
-        norms = [torch.empty((n,), dtype=torch.int16, device=device) for _ in range(copies)]
-        st = RateState(rate, rot, cb, index, P, codes, norms)
+        codes = [torch.empty((n, P), dtype=torch.uint8, device=device) for _ in range(ncopies)]
+        norms = [torch.empty((n,), dtype=torch.int16, device=device) for _ in range(ncopies)]
+        return RateState(rate, rot, cb, index, P, codes, norms)
+
+    step = [rate_state(r, copies) for r in step_rates]
+    for st in step:
         for c in range(copies):  # valid records everywhere before timing
             for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
-                fq.fq_encode(xs[c][sl], rot[t], cb, rate.k, rate.N, codes=codes[c][sl],
-                             norms=norms[c][sl], search_index=index)
-        states.append(st)
-    ys = [torch.empty((n, d), dtype=torch.float16, device=device) for _ in range(copies)]
+                fq.fq_encode(xs[c][sl], st.rot[t], st.cb, st.rate.k, st.rate.N,
+                             codes=st.codes[c][sl], norms=st.norms[c][sl], search_index=st.index)
+    extra = [rate_state(r, 1) for r in extra_rates]
+    ys = [torch.empty((n, d), dtype=tdtype, device=device) for _ in range(copies)]
     torch.cuda.synchronize()
-    return shape, host, xs, ys, states
+    return CodecRun(w, shape, host, xs, ys, step, extra, copies)
 
 
-def codec_launches(fq, shape, xs, ys, states, c, prev):
+def codec_launches(fq, run, c, prev):
     """The launches of one step on copy c (decode reads the records of copy `prev`).  Yields
-    (label, kind, algorithmic bytes, fp16-equivalent bytes, launch thunk)."""
-    n, d = shape.n, shape.d
+    (label, kind, algorithmic bytes, fp16-equivalent bytes, vectors, launch thunk)."""
+    n, d = run.shape.n, run.shape.d
     half = n // 2
-    for st in states:
+    xs, ys = run.xs, run.ys
+    for st in run.step:
         r = st.rate
         for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
             nv = sl.stop - sl.start
             xb = xs[c].element_size() * d
-            yield (f"encode_{r.label}", "encode", nv * (xb + st.P + 2), nv * 2 * d,
+            yield (f"encode_{r.label}", "encode", nv * (xb + st.P + 2), nv * 2 * d, nv,
                    lambda st=st, t=t, sl=sl: fq.fq_encode(
                        xs[c][sl], st.rot[t], st.cb, st.rate.k, st.rate.N, codes=st.codes[c][sl],
                        norms=st.norms[c][sl], search_index=st.index))
-            yield (f"decode_{r.label}", "decode", nv * (st.P + 2 + 2 * d), nv * 2 * d,
+            yield (f"decode_{r.label}", "decode", nv * (st.P + 2 + 2 * d), nv * 2 * d, nv,
                    lambda st=st, t=t, sl=sl: fq.fq_decode(
                        st.codes[prev][sl], st.norms[prev][sl], st.rot[t], st.cb, d, st.rate.k,
                        st.rate.N, y=ys[c][sl]))
 
+
+def extra_launches(fq, run, c):
+    n, d = run.shape.n, run.shape.d
+    half = n // 2
+    for st in run.extra:
+        for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
+            nv = sl.stop - sl.start
+            yield (f"encode_{st.rate.label}", "encode", nv * (2 * d + st.P + 2), nv * 2 * d, nv,
+                   lambda st=st, t=t, sl=sl: fq.fq_encode(
+                       run.xs[c][sl], st.rot[t], st.cb, st.rate.k, st.rate.N,
+                       codes=st.codes[0][sl], norms=st.norms[0][sl], search_index=st.index))
+
+
+class GraphTimer:
+    """CUDA-graph capture on a side stream and CUDA-event timing on the launching stream."""
+
+    def __init__(self, torch, device, dist):
+        self.torch, self.dist, self.device = torch, dist, device
+        self.stream = torch.cuda.current_stream()
+        self.side = torch.cuda.Stream(device)
+        self.side.wait_stream(self.stream)
+
+    def capture(self, fns):
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.stream(self.side):
+            with self.torch.cuda.graph(g, stream=self.side):
+                for fn in fns:
+                    fn()
+        return g
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+        self.torch.cuda.synchronize()
+
+    def time(self, graphs, reps):
+        """ms for `reps` replays cycling over `graphs` (max over ranks)."""
+        self.barrier()
+        e0 = self.torch.cuda.Event(enable_timing=True)
+        e1 = self.torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for i in range(reps):
+            graphs[i % len(graphs)].replay()
+        e1.record(self.stream)
+        self.barrier()
+        return max_over_ranks(self.torch, self.dist, e0.elapsed_time(e1), self.device)
+
+    def adaptive_reps(self, graphs, target_s=0.25, lo=2, hi=50):
+        """Replays that fill about target_s (measured on one replay of every graph)."""
+        ms = self.time(graphs, len(graphs)) / len(graphs)
+        return max(lo, min(hi, int(target_s * 1e3 / max(ms, 1e-3))))
+
+
+def kernel_table(timer, fq, run, launches_of, hbm):
+    """Per-label device time: a graph of every launch of one label over all copies, replayed."""
+    per = {}
+    meta = [m[:5] for m in launches_of(0)]
+    for lab in dict.fromkeys(m[0] for m in meta):
+        fns = [fn for c in range(run.copies) for (l, *_, fn) in launches_of(c) if l == lab]
+        g = timer.capture(fns)
+        reps = timer.adaptive_reps([g])
+        ms = timer.time([g], reps) / (reps * len(fns))
+        _, kind, ab, _, nv = next(m for m in meta if m[0] == lab)
+        per_step = sum(1 for m in meta if m[0] == lab)
+        gbs = ab / (ms * 1e-3) / 1e9
+        per[lab] = {"ms": ms, "per_step": per_step, "alg_bytes": ab, "kind": kind, "vectors": nv,
+                    "GBps": gbs, "frac": gbs / hbm}
+        del g
+    return per
+
+
+def kernels_json(per, with_share=True):
+    tot = sum(v["ms"] * v["per_step"] for v in per.values())
+    out = {}
+    for lab, s in per.items():
+        o = {"avg_us": round(1e3 * s["ms"], 2), "vectors_per_launch": s["vectors"],
+             "Gvec_s": round(s["vectors"] / (s["ms"] * 1e-3) / 1e9, 3),
+             "GBps_alg": round(s["GBps"], 1), "frac": round(s["frac"], 4)}
+        if with_share:
+            o["share"] = round(s["ms"] * s["per_step"] / tot, 3)
+        out[lab] = o
+    return out
+
+
+def time_codec_step(timer, fq, run, steps, warmup, clocks=None):
+    """(total ms over `steps` step replays, step graphs' metadata).  The step graphs cycle over
+    the input copies; decode of copy c reads the records of copy c - 1."""
+    copies = run.copies
+    for c in range(copies):  # one eager pass (tables, attributes) before capture
+        for *_, fn in codec_launches(fq, run, c, (c - 1) % copies):
+            fn()
+    timer.torch.cuda.synchronize()
+    graphs = [timer.capture([fn for *_, fn in codec_launches(fq, run, c, (c - 1) % copies)])
+              for c in range(copies)]
+    meta = [m[:5] for m in codec_launches(fq, run, 0, copies - 1)]
+    for i in range(warmup):
+        graphs[i % copies].replay()
+    timer.barrier()
+    if clocks is None:
+        ms = timer.time(graphs, steps)
+    else:
+        with clocks:
+            ms = timer.time(graphs, steps)
+    del graphs
+    return ms, meta
+
+
+# ----------------------------------------------------------------------------- attention
 
 def attn_state(torch, fq, device, copies, rank):
     w = wl.ATTN
@@ -254,11 +444,18 @@ def attn_state(torch, fq, device, copies, rank):
     ck = torch.from_numpy(tables.codebook(dpk, w.k_rate.k, w.k_rate.N)).to(device)
     cv = torch.from_numpy(tables.codebook(dpv, w.v_rate.k, w.v_rate.N)).to(device)
     q = torch.from_numpy(wl.attn_queries(w)).to(device)
-    kx = torch.from_numpy(wl.attn_kv(w, "K").reshape(-1, w.d)).to(device)
-    vx = torch.from_numpy(wl.attn_kv(w, "V").reshape(-1, w.d)).to(device)
-    kc, kn = fq.fq_encode(kx, rk, ck, w.k_rate.k, w.k_rate.N)
-    vc, vn = fq.fq_encode(vx, rv, cv, w.v_rate.k, w.v_rate.N)
-    del kx, vx
+    kx = torch.from_numpy(wl.attn_kv(w, "K")).to(device)
+    vx = torch.from_numpy(wl.attn_kv(w, "V")).to(device)
+    kc, kn = fq.fq_encode(kx.reshape(-1, w.d), rk, ck, w.k_rate.k, w.k_rate.N)
+    vc, vn = fq.fq_encode(vx.reshape(-1, w.d), rv, cv, w.v_rate.k, w.v_rate.N)
+    # sanity metric: exact softmax attention over the uncompressed fp16 cache (plain PyTorch,
+    # fp32), to compare the compressed step's output with by cosine similarity
+    G = w.hq // w.hkv
+    qf = q.float().reshape(w.batch, w.hkv, G, w.d)
+    s = torch.einsum("bhgd,bhtd->bhgt", qf, kx.float()) / math.sqrt(w.d)
+    exact = torch.einsum("bhgt,bhtd->bhgd", torch.softmax(s, dim=-1), vx.float())
+    exact = exact.reshape(w.batch, w.hq, w.d)
+    del kx, vx, s
     shp = (w.batch, w.hkv, w.tokens)
     kcs = [kc.reshape(*shp, -1).clone() for _ in range(copies)]
     kns = [kn.reshape(shp).clone() for _ in range(copies)]
@@ -273,10 +470,48 @@ def attn_state(torch, fq, device, copies, rank):
         fq.fq_attn_decode(q, kcs[c], kns[c], w.k_rate.k, w.k_rate.N, rk, ck, vcs[c], vns[c],
                           w.v_rate.k, w.v_rate.N, rv, cv, scale=1 / math.sqrt(w.d), out=out,
                           workspace=ws)
-    return launch, step_bytes
+
+    def cosine():
+        launch(0)
+        torch.cuda.synchronize()
+        cs = torch.nn.functional.cosine_similarity(out, exact, dim=-1)
+        return float(cs.mean()), float(cs.min())
+    return launch, step_bytes, cosine
+
+
+def attn_bench(torch, fq, timer, device, rank, hbm):
+    launch, attn_bytes, cosine = attn_state(torch, fq, device, 4, rank)
+    for c in range(4):
+        launch(c)
+    torch.cuda.synchronize()
+    graphs = [timer.capture([lambda c=c: launch(c)]) for c in range(4)]
+    for g in graphs:
+        g.replay()
+    reps = timer.adaptive_reps(graphs, target_s=0.25, lo=20, hi=2000)
+    us = timer.time(graphs, reps) * 1e3 / reps
+    del graphs
+    cmean, cmin = cosine()
+    gbs = attn_bytes / (us * 1e-6) / 1e9
+    return {"workload": wl.ATTN.name, "us_per_step": round(us, 2), "bytes_per_step": attn_bytes,
+            "reps": reps,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4)},
+            "launches_per_step": 2,
+            "cosine_vs_exact_fp16_attention": {"mean": round(cmean, 5), "min": round(cmin, 5)}}
 
 
 # ----------------------------------------------------------------------------- arms
+
+def compression(w, fq):
+    out = {}
+    d = w.cache.d
+    for r in w.rates:
+        P = fq.fq_payload_bytes(d, r.k, r.N)
+        b = math.log2(r.N) / r.k
+        out[r.label] = {"bits_per_coord": round(b, 4), "pages_16_over_b": round(16 / b, 2),
+                        "true_fp16_over_record": round(2 * d / (P + 2), 2)}
+    return out
+
 
 def run_gpu(args):
     import torch
@@ -292,163 +527,118 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    w = pick_workload(args)
-    shape0 = w.cache
-    step_bytes_est = shape0.n * (shape0.d * 2) * 3 * len(w.rates)
-    copies = max(2, math.ceil(2 * L2_BYTES / max(step_bytes_est, 1)) + 1)
-    copies = min(copies, 8)
-    shape, host, xs, ys, states = build_codec_state(torch, fq, w, rank, copies, device)
-    attn_launch, attn_bytes = attn_state(torch, fq, device, 4, rank) if not args.no_attn else (None, 0)
-    n_launch = sum(1 for _ in codec_launches(fq, shape, xs, ys, states, 0, 0))
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    stream = torch.cuda.current_stream()
-    # The timed region replays CUDA graphs of the step's C-ABI calls (one graph per input copy):
-    # the kernels, arguments and order are those of the eager calls, without the host-side
-    # launch latency between them.
-    side = torch.cuda.Stream(device)
-    side.wait_stream(stream)
-
-    def capture(fns):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(g, stream=side):
-                for fn in fns:
-                    fn()
-        return g
-
-    for c in range(copies):  # one eager pass (tables, attributes) before capture
-        for *_, fn in codec_launches(fq, shape, xs, ys, states, c, (c - 1) % copies):
-            fn()
-    torch.cuda.synchronize()
-    step_graphs = [capture([fn for *_, fn in codec_launches(fq, shape, xs, ys, states, c,
-                                                             (c - 1) % copies)])
-                   for c in range(copies)]
-    meta = [(lab, kind, ab, eb) for lab, kind, ab, eb, _ in
-            codec_launches(fq, shape, xs, ys, states, 0, copies - 1)]
-    torch.cuda.synchronize()
-    for i in range(args.warmup):
-        step_graphs[i % copies].replay()
-    barrier()
-    with ClockSampler(local) as clk:
-        barrier()
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for i in range(args.steps):
-            step_graphs[i % copies].replay()
-        t_end.record(stream)
-        barrier()
-    total_ms = max_over_ranks(torch, dist, t_start.elapsed_time(t_end), device)
-    # per-kernel device time: a graph of every launch of one kind over all copies, replayed
-    per = {}
-    reps = max(5, min(50, args.steps // copies))
-    for lab in dict.fromkeys(m[0] for m in meta):
-        fns = [fn for c in range(copies) for l, *_, fn in
-               codec_launches(fq, shape, xs, ys, states, c, (c - 1) % copies) if l == lab]
-        g = capture(fns)
-        g.replay()
-        barrier()
-        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        k0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        k1.record(stream)
-        barrier()
-        ms = k0.elapsed_time(k1) / (reps * len(fns))
-        ab, kind = next((m[2], m[1]) for m in meta if m[0] == lab)
-        per_step = sum(1 for m in meta if m[0] == lab)
-        per[lab] = {"ms": ms, "per_step": per_step, "alg_bytes": ab, "kind": kind}
-        del g
-    step_eq = sum(eb for _, _, _, eb in meta)
-    value = whole_job_rate(world, step_eq, args.steps, total_ms)
     hbm, hbm_src = peaks()
+    timer = GraphTimer(torch, device, dist)
+    w = pick_workload(args)
+
+    # ---- headline: the step over the named workload, with clocks sampled during the region
+    run = build_codec_run(torch, fq, w, rank, device)
+    clk = ClockSampler(torch, local)
+    total_ms, meta = time_codec_step(timer, fq, run, args.steps, args.warmup, clocks=clk)
+    step_eq = sum(m[3] for m in meta)
+    value = whole_job_rate(world, step_eq, args.steps, total_ms)
+    per = kernel_table(timer, fq, run, lambda c: codec_launches(fq, run, c, (c - 1) % run.copies),
+                       hbm)
+    extra = kernel_table(timer, fq, run, lambda c: extra_launches(fq, run, c), hbm) \
+        if run.extra else {}
     dom_lab = max(per, key=lambda k: per[k]["ms"] * per[k]["per_step"])
     dom = per[dom_lab]
-    achieved = dom["alg_bytes"] / (dom["ms"] * 1e-3) / 1e9
-    tot_share = sum(v["ms"] * v["per_step"] for v in per.values())
-    kernels = {lab: {"avg_us": round(1e3 * s_["ms"], 2),
-                     "GBps_alg": round(s_["alg_bytes"] / (s_["ms"] * 1e-3) / 1e9, 1),
-                     "share": round(s_["ms"] * s_["per_step"] / tot_share, 3)}
-               for lab, s_ in per.items()}
+    traffic = profiled_traffic(w.name, dom_lab, run.shape.d, dom["vectors"])
+    step_rates, extra_rates = step_and_extra_rates(w)
     result = {
-        "metric": "KV encode/decode GB/s (fp16-equiv) & % of roofline; fused attn us/step",
-        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16->u8/fp32",
-        "data": "synthetic (seeded; GPT-2-small-shaped KV cache recipe, no weights)",
-        "config": {"workload": w.name, "vectors_per_gpu": shape.n, "d": shape.d,
-                   "rates": [r.label for r in w.rates], "decode_out": "fp16",
-                   "l2": f"inputs rotate over {copies} copies (>= 2x L2 between reuses)",
-                   "step": "encode K,V + decode K,V per rate",
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16->u8->fp16",
+        "data": "synthetic (seeded KV-cache recipe of the pages' workloads, no model weights)",
+        "config": {"workload": w.name, "vectors_per_gpu": run.shape.n, "d": run.shape.d,
+                   "step_rates": [r.label for r in step_rates],
+                   "extra_kernels": [f"encode_{r.label}" for r in extra_rates],
+                   "io": "fp16 in -> u8 records + fp16 norms -> fp16 out",
+                   "math": "fp32 (tensor-core operands split into fp16 hi + lo)",
+                   "l2": (f"inputs {run.copies} copies, >= 2x L2 between reuses" if run.copies > 1
+                          else "inputs larger than 2x L2 (no reuse within a step)"),
+                   "step": "encode K,V + decode K,V (fp16 out) per step rate",
                    "launch": "CUDA graph replay of the step's C-ABI calls"},
-        "roofline": {"bound": "hbm", "kernel": dom_lab, "achieved": round(achieved, 1),
-                     "peak": hbm, "peak_source": hbm_src, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": profiled_traffic(dom_lab),
-                     "alg_bytes_per_launch": dom["alg_bytes"]},
-        "kernels": kernels,
-        "gpu_launches": None,
+        "roofline": {"bound": "hbm", "kernel": dom_lab,
+                     "achieved": round(dom["GBps"], 1), "peak": hbm, "peak_source": hbm_src,
+                     "unit": "GB/s", "frac": round(dom["frac"], 4), "traffic": traffic,
+                     "alg_bytes_per_launch": dom["alg_bytes"],
+                     "alg_bytes_per_vector": dom["alg_bytes"] // dom["vectors"]},
+        "kernels": kernels_json(per),
+        "extra_kernels": kernels_json(extra, with_share=False),
+        "gpu_launches": len(meta) * args.steps,
         "clocks": clk.summary(),
+        "compression": compression(w, fq),
     }
-    launches_per_step = len(meta)
-    gpu_launches = launches_per_step * args.steps
-    # fused attention step
-    if attn_launch:
-        for c in range(4):
-            attn_launch(c)
-        torch.cuda.synchronize()
-        agraphs = [capture([lambda c=c: attn_launch(c)]) for c in range(4)]
-        areps = max(20, args.steps // 10)
-        for i in range(4):
-            agraphs[i].replay()
-        barrier()
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for i in range(areps):
-            agraphs[i % 4].replay()
-        a1.record(stream)
-        barrier()
-        us = max_over_ranks(torch, dist, a0.elapsed_time(a1), device) * 1e3 / areps
-        result["attn"] = {"workload": wl.ATTN.name, "us_per_step": round(us, 2),
-                          "bytes_per_step": attn_bytes,
-                          "roofline": {"bound": "hbm", "achieved": round(attn_bytes / (us * 1e-6) / 1e9, 1),
-                                       "peak": hbm, "unit": "GB/s",
-                                       "frac": round(attn_bytes / (us * 1e-6) / 1e9 / hbm, 4)},
-                          "launches_per_step": 2}
-        del agraphs
-    del step_graphs
-    result["gpu_launches"] = gpu_launches
-    # end to end through the public API with pinned host buffers
+    # ---- end to end through the public API with pinned host buffers (headline workload)
     if not args.no_e2e:
-        result["e2e"] = e2e(torch, fq, shape, host, states, args, device, world, dist)
+        result["e2e"] = e2e(torch, fq, run, args, device, world, dist)
+    host_sample = None
+    if rank == 0 and not args.no_cpu:
+        host_sample = cpu_sample_rows(run.shape)
+        host_sample = (host_sample, run.host[host_sample])
+    del run
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads (their own steps), reported under "configs"
+    if not args.no_configs and not args.tokens:
+        result["configs"] = {}
+        for key, cw in WORKLOADS.items():
+            if cw is WORKLOADS[args.workload]:
+                continue
+            r2 = build_codec_run(torch, fq, cw, rank, device)
+            steps2 = max(20, args.steps)
+            ms2, meta2 = time_codec_step(timer, fq, r2, steps2, max(3, args.warmup))
+            per2 = kernel_table(timer, fq, r2,
+                                lambda c: codec_launches(fq, r2, c, (c - 1) % r2.copies), hbm)
+            v2 = whole_job_rate(world, sum(m[3] for m in meta2), steps2, ms2)
+            result["configs"][cw.name] = {
+                "value": round(v2, 2), "unit": "GB/s", "steps": steps2,
+                "ms_per_step": round(ms2 / steps2, 4), "vectors_per_gpu": r2.shape.n,
+                "rates": [r.label for r in cw.rates], "kernels": kernels_json(per2),
+                "compression": compression(cw, fq)}
+            del r2
+            torch.cuda.empty_cache()
+
+    # ---- fused attention step
+    if not args.no_attn:
+        result["attn"] = attn_bench(torch, fq, timer, device, rank, hbm)
+    bad = fq.fq_wait_status(clear=True)
+    if bad:
+        raise RuntimeError(f"{bad} CTAs gave up a bounded wait during the bench")
     if rank == 0:
-        result["cpu_baseline"] = cpu_baseline(w, args) if not args.no_cpu else None
+        if host_sample is not None:
+            result["cpu_baseline"] = cpu_baseline(w, args, sample=host_sample)
         print(json.dumps(result), flush=True)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
 
 
-def e2e(torch, fq, shape, host, states, args, device, world, dist, chunks=8):
+def e2e(torch, fq, run, args, device, world, dist, chunks=8):
     """Same metric through the public API with host buffers.  Every step copies the pinned host
     cache in, encodes, copies the records out, copies them back in, decodes and copies the fp16
-    result out, for each rate.  The step runs in row chunks (each entirely K or V) over three
-    CUDA streams (upload, kernels, download) so that uploads, downloads and kernels overlap.  The step's calls are captured once as a CUDA graph and replayed, as in
-    the device-resident measurement; every byte still crosses the host link in every step."""
+    result out, for each step rate.  The step runs in row chunks (each entirely K or V) over three
+    CUDA streams (upload, kernels, download) so that uploads, downloads and kernels overlap.  The
+    step's calls are captured once as a CUDA graph and replayed, as in the device-resident
+    measurement; every byte still crosses the host link in every step."""
+    shape, states = run.shape, run.step
     n, d = shape.n, shape.d
     half = n // 2
     per = half // (chunks // 2)
     assert per * chunks == n, "chunks must split the K and V halves evenly"
-    xh = torch.from_numpy(host).pin_memory()
-    xd = torch.empty_like(xh, device=device)
+    xh = torch.from_numpy(run.host).pin_memory()
+    xd = run.xs[0]
     rec_h = [(torch.empty((n, st.P), dtype=torch.uint8).pin_memory(),
               torch.empty((n,), dtype=torch.int16).pin_memory()) for st in states]
+    rec_out = [(torch.empty((n, st.P), dtype=torch.uint8, device=device),
+                torch.empty((n,), dtype=torch.int16, device=device)) for st in states]
+    rec_in = [(torch.empty((n, st.P), dtype=torch.uint8, device=device),
+               torch.empty((n,), dtype=torch.int16, device=device)) for st in states]
     yh = [torch.empty((n, d), dtype=torch.float16).pin_memory() for _ in states]
-    yd = [torch.empty((n, d), dtype=torch.float16, device=device) for _ in states]
+    yd = [run.ys[0]] + [torch.empty((n, d), dtype=torch.float16, device=device)
+                        for _ in states[1:]]
     cs, su, sc, sd = (torch.cuda.Stream(device) for _ in range(4))
 
     def rows(j):
@@ -463,7 +653,7 @@ def e2e(torch, fq, shape, host, states, args, device, world, dist, chunks=8):
         # Enqueued from cs (fork and join).  One stream per copy direction, each in data-flow
         # order with a lag of one chunk, so that no copy waits behind a later chunk's copies:
         #   su (upload):   x0 x1 r0 x2 r1 ...    (r = records back in)
-        #   sc (kernels):  e0 e1 d0 e2 d1 ...    (e = encode, d = decode; both rates)
+        #   sc (kernels):  e0 e1 d0 e2 d1 ...    (e = encode, d = decode; every step rate)
         #   sd (download): o0 o1 y0 o2 y1 ...    (o = records out, y = fp16 result)
         e0 = mark(cs)
         for s_ in (su, sc, sd):
@@ -479,31 +669,29 @@ def e2e(torch, fq, shape, host, states, args, device, world, dist, chunks=8):
                 sl, _ = rows(j - 1)
                 su.wait_event(ev_out[j - 1])
                 with torch.cuda.stream(su):
-                    for r, st in enumerate(states):
-                        ch, nh = rec_h[r]
-                        st.codes[1][sl].copy_(ch[sl], non_blocking=True)
-                        st.norms[1][sl].copy_(nh[sl], non_blocking=True)
+                    for r in range(len(states)):
+                        rec_in[r][0][sl].copy_(rec_h[r][0][sl], non_blocking=True)
+                        rec_in[r][1][sl].copy_(rec_h[r][1][sl], non_blocking=True)
                 ev_in[j - 1] = mark(su)
             if j < chunks:
                 sl, t = rows(j)
                 sc.wait_event(ev_x[j])
-                for st in states:
+                for r, st in enumerate(states):
                     fq.fq_encode(xd[sl], st.rot[t], st.cb, st.rate.k, st.rate.N,
-                                 codes=st.codes[0][sl], norms=st.norms[0][sl],
+                                 codes=rec_out[r][0][sl], norms=rec_out[r][1][sl],
                                  search_index=st.index, stream=sc)
                 ev_enc[j] = mark(sc)
                 sd.wait_event(ev_enc[j])
                 with torch.cuda.stream(sd):
-                    for r, st in enumerate(states):
-                        ch, nh = rec_h[r]
-                        ch[sl].copy_(st.codes[0][sl], non_blocking=True)
-                        nh[sl].copy_(st.norms[0][sl], non_blocking=True)
+                    for r in range(len(states)):
+                        rec_h[r][0][sl].copy_(rec_out[r][0][sl], non_blocking=True)
+                        rec_h[r][1][sl].copy_(rec_out[r][1][sl], non_blocking=True)
                 ev_out[j] = mark(sd)
             if j >= 1:
                 sl, t = rows(j - 1)
                 sc.wait_event(ev_in[j - 1])
                 for r, st in enumerate(states):
-                    fq.fq_decode(st.codes[1][sl], st.norms[1][sl], st.rot[t], st.cb, d,
+                    fq.fq_decode(rec_in[r][0][sl], rec_in[r][1][sl], st.rot[t], st.cb, d,
                                  st.rate.k, st.rate.N, y=yd[r][sl], stream=sc)
                 ev_dec[j - 1] = mark(sc)
                 sd.wait_event(ev_dec[j - 1])
@@ -523,20 +711,25 @@ def e2e(torch, fq, shape, host, states, args, device, world, dist, chunks=8):
     with torch.cuda.graph(graph, stream=cs):
         step()
     torch.cuda.synchronize()
-    for _ in range(max(3, args.warmup // 10)):
+    for _ in range(3):
         graph.replay()
     torch.cuda.synchronize()
     # the overlapped step must deliver exactly what a plain decode of its records gives
     for r, st in enumerate(states):
         ref = torch.empty((n, d), dtype=torch.float16, device=device)
         for t, sl in (("K", slice(0, half)), ("V", slice(half, n))):
-            fq.fq_decode(st.codes[1][sl], st.norms[1][sl], st.rot[t], st.cb, d, st.rate.k,
+            fq.fq_decode(rec_in[r][0][sl], rec_in[r][1][sl], st.rot[t], st.cb, d, st.rate.k,
                          st.rate.N, y=ref[sl])
         if not torch.equal(ref.cpu(), yh[r]):
             raise RuntimeError(f"overlapped end-to-end step disagrees with a plain decode "
                                f"({st.rate.label})")
+        del ref
     torch.cuda.synchronize()
-    reps = max(5, min(50, args.steps // 20))
+    g1 = time.perf_counter()
+    graph.replay()
+    torch.cuda.synchronize()
+    one = time.perf_counter() - g1
+    reps = max(3, min(20, int(1.0 / max(one, 1e-4))))
     if dist is not None:
         dist.barrier()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -554,32 +747,80 @@ def e2e(torch, fq, shape, host, states, args, device, world, dist, chunks=8):
                        "in data-flow order, one CUDA graph per step"}
 
 
-def cpu_baseline(w, args, budget_s: float = 12.0):
-    """The CPU oracle, as it stands, timed on this host on a bounded sample of the workload
-    (single BLAS thread)."""
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_sample_rows(shape, count=4096):
+    """The CPU baseline's sample: rows drawn from the first key slab and the first value slab (so
+    that the reference arm regenerates two slabs only, not the whole cache)."""
+    per = shape.slab_vectors
+    first_v = shape.batch * shape.layers * per
+    rng = np.random.default_rng(0)
+    k = rng.choice(per, size=min(count // 2, per), replace=False)
+    v = first_v + rng.choice(per, size=min(count // 2, per), replace=False)
+    return np.sort(np.concatenate([k, v]))
+
+
+def _oracle_warm(_):
+    """Imports the oracle in a pool process before the timed window opens."""
+    from oracle import fq_oracle  # noqa: F401
+    from random_access_kv_fq_b200 import tables  # noqa: F401
+    return 0
+
+
+def _oracle_worker(job):
+    """One host process: encode + pack + decode of its rows with the oracle, repeated until the
+    deadline (wall-clock time.time()).  Returns (fp16-equivalent bytes done, seconds)."""
+    x, rates, d, deadline, call_rows = job
     from threadpoolctl import threadpool_limits
     from oracle import fq_oracle as fo
     from random_access_kv_fq_b200 import tables
-    shape = w.cache
-    rng = np.random.default_rng(0)
-    sample = np.sort(rng.choice(shape.n, size=min(2048, shape.n), replace=False))
-    x = wl.rows_of(shape, sample)
-    done_eq = 0
-    t0 = time.perf_counter()
+    done = 0
+    t0 = time.time()
     with threadpool_limits(1):
-        while time.perf_counter() - t0 < budget_s:
-            for rate in w.rates:
-                dp = fo.padded_dim(shape.d, rate.k)
-                rot = tables.rotation(dp, wl.ROT_SEED_K)
-                cb = tables.codebook(dp, rate.k, rate.N)
-                enc = fo.encode(x, rot, cb, rate.k)
-                codes = fo.pack(enc.idx, rate.N)
-                fo.decode(codes, enc.norms, rot, cb, shape.d, rate.k, rate.N)
-                done_eq += 2 * x.shape[0] * 2 * shape.d
-    el = time.perf_counter() - t0
-    return {"value": round(done_eq / el / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{x.shape[0]} sampled vectors of {w.name}, encode+pack+decode at every "
-                      f"rate, repeated for {el:.1f} s (fp64 NumPy, 1 thread)"}
+        while time.time() < deadline:
+            for (k, N) in rates:
+                dp = fo.padded_dim(d, k)
+                rot, cb = tables.rotation(dp, wl.ROT_SEED_K), tables.codebook(dp, k, N)
+                for s in range(0, x.shape[0], call_rows):
+                    xc = x[s:s + call_rows]
+                    enc = fo.encode(xc, rot, cb, k)
+                    fo.decode(fo.pack(enc.idx, N), enc.norms, rot, cb, d, k, N)
+                    done += 2 * xc.shape[0] * 2 * d
+                    if time.time() >= deadline:
+                        break
+    return done, time.time() - t0
+
+
+def cpu_baseline(w, args, budget_s: float = 12.0, sample=None):
+    """The CPU oracle, as it stands, on a bounded sample of the workload, one process per host
+    core (spawned), each with one BLAS thread: fp16-equivalent GB/s of encode + pack + decode at
+    the step's rates (the exact brute-force search: the oracle's definition of the encoder)."""
+    import multiprocessing as mp
+    shape = w.cache
+    if sample is None:
+        rows = cpu_sample_rows(shape)
+        sample = (rows, wl.rows_of(shape, rows))
+    rows, x = sample
+    step_rates, _ = step_and_extra_rates(w)
+    rates = [(r.k, r.N) for r in step_rates]
+    cores = len(os.sched_getaffinity(0))
+    call_rows = 16 if shape.d == 128 else 256
+    parts = [x[i::cores] for i in range(cores)]
+    parts = [p for p in parts if p.shape[0]]
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(len(parts)) as pool:
+        # workers start and import the oracle before the clock: all share one deadline
+        pool.map(_oracle_warm, range(len(parts)), chunksize=1)
+        deadline = time.time() + budget_s
+        res = pool.map(_oracle_worker, [(p, rates, shape.d, deadline, call_rows) for p in parts])
+    done = sum(r[0] for r in res)
+    el = max(r[1] for r in res)
+    return {"value": round(done / el / 1e9, 6), "unit": "GB/s", "cores": len(parts),
+            "kind": "oracle",
+            "sample": f"{x.shape[0]} vectors of {w.name} (first key and value slabs), "
+                      f"encode+pack+decode at {[r.label for r in step_rates]} with the oracle's "
+                      f"brute-force encoder, repeated for {el:.1f} s in {len(parts)} spawned "
+                      f"processes (fp64 NumPy, 1 BLAS thread each)"}
 
 
 def run_reference(args):
@@ -588,12 +829,12 @@ def run_reference(args):
         return
     w = pick_workload(args)
     cb = cpu_baseline(w, args, budget_s=max(3.0, min(20.0, 2.0 * args.steps)))
-    line = {"impl": "reference", "metric": "KV encode/decode GB/s (fp16-equiv) & % of roofline; "
-            "fused attn us/step", "value": cb["value"], "unit": "GB/s",
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
             "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "rates": [r.label for r in w.rates]},
+            "config": {"workload": w.name,
+                       "step_rates": [r.label for r in step_and_extra_rates(w)[0]]},
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -603,10 +844,11 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="fibquant", choices=["fibquant", "reference"])
-    ap.add_argument("--workload", default="gpt2", choices=list(WORKLOADS))
+    ap.add_argument("--workload", default="large", choices=list(WORKLOADS))
+    ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--no-attn", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

@@ -170,12 +170,26 @@ def slabs(shape: CacheShape) -> Iterator[tuple[int, np.ndarray]]:
                 row += s.shape[0]
 
 
-def cache(shape: CacheShape) -> np.ndarray:
-    """The whole flat [n, d] K+V cache (host memory)."""
+def cache(shape: CacheShape, workers: int = 1) -> np.ndarray:
+    """The whole flat [n, d] K+V cache (host memory).  Slabs are independent, so `workers`
+    threads may draw them at once (NumPy's generators release the GIL); the result does not
+    depend on `workers`."""
     dt = np.float16 if shape.dtype == "f16" else np.float32
     out = np.empty((shape.n, shape.d), dtype=dt)
-    for row, s in slabs(shape):
-        out[row:row + s.shape[0]] = s
+    jobs = [(tensor, b, layer) for tensor in ("K", "V") for b in range(shape.batch)
+            for layer in range(shape.layers)]
+
+    def fill(i):
+        s = slab(shape, *jobs[i])
+        out[i * s.shape[0]:(i + 1) * s.shape[0]] = s
+
+    if workers <= 1:
+        for i in range(len(jobs)):
+            fill(i)
+    else:
+        import concurrent.futures as cf
+        with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(fill, range(len(jobs))))
     return out
 
 
