@@ -30,8 +30,8 @@
  *   - Errors are returned as fq_status from host-side validation before anything is enqueued,
  *     or FQ_ERR_CUDA when a launch fails.  Nothing aborts or throws across the ABI.
  *   - n = 0 (or T = 0 in attention) is a valid no-op returning FQ_OK.
- *   - Limits: 1 <= d <= 256, 1 <= k <= 8, k <= d, N a power of two in [2, 65536]; other
- *     values return FQ_ERR_UNSUPPORTED.  Non-finite inputs are a precondition violation and
+ *   - Limits: 1 <= d <= 256, 1 <= k <= d, N a power of two in [2, 65536]; other values
+ *     return FQ_ERR_UNSUPPORTED.  Non-finite inputs are a precondition violation and
  *     are not detected.
  *   - Rotation `rot`: d' x d' fp32, row-major, z = rot * pad(x) (rows = output coordinates).
  *     Codebook `codebook`: N x k fp32, row-major.  Both are plain input data; the library
@@ -62,8 +62,17 @@ typedef enum { FQ_F16 = 0, FQ_F32 = 1 } fq_dtype;
 /* Search-index kinds for fq_build_search_index. */
 typedef enum {
   FQ_INDEX_EXACT = 0, /* conservative candidate lists: identical results to brute force */
-  FQ_INDEX_TOPC = 1   /* Cartesian grid, c codewords nearest each cell centre (approximate) */
+  FQ_INDEX_TOPC = 1,  /* Cartesian grid, c codewords nearest each cell centre (approximate) */
+  FQ_INDEX_TENSOR = 2 /* the codebook as tensor-core operand tiles, for half- and full-vector
+                         codes (k = 32 or 64): brute-force GEMM search, brute-force results */
 } fq_index_kind;
+
+/* Decoder rescale rules (Block Sphere VQ notes, key design 3), for fq_decode_rescaled. */
+typedef enum {
+  FQ_RESCALE_PLAIN = 0,    /* S = 1: the plain decoder, as fq_decode */
+  FQ_RESCALE_MSE = 1,      /* S = rho / |zbar|^2: least squared reconstruction error */
+  FQ_RESCALE_UNBIASED = 2  /* S = 1 / rho: unbiased inner products */
+} fq_rescale_rule;
 
 /* ABI version of this header (bumped on any incompatible change). */
 int fq_abi_version(void);
@@ -106,6 +115,67 @@ fq_status fq_decode(const uint8_t* codes, const uint16_t* norms, int64_t n, int 
                     void* stream);
 
 /*
+ * fq_decode_gather - random access (summary sec. 1: every record sits at a fixed address, so
+ * any token decodes alone): y[i] = decode of record token_ids[i], for a token list in any order
+ * with repeats allowed.
+ *   codes, norms   a plane of n_records records (as produced by fq_encode).
+ *   token_ids      [n_ids] int64 device array, 8-byte aligned.  An id outside [0, n_records)
+ *                  reads nothing and gives a row of NaN (ids live on the device, so they are
+ *                  checked there, not on the host).
+ *   y              [n_ids, d] output, fp32 or fp16 (y_type), aligned as in fq_decode.
+ * Results equal fq_decode of the listed records.
+ */
+fq_status fq_decode_gather(const uint8_t* codes, const uint16_t* norms, int64_t n_records,
+                           const int64_t* token_ids, int64_t n_ids, int d, int k, int N,
+                           const float* rot, const float* codebook, void* y, fq_dtype y_type,
+                           void* stream);
+
+/*
+ * fq_encode_rho - fq_encode that also stores, per vector, the alignment rho = <z, zbar> of the
+ * unit rotated vector z with its reconstruction zbar (the concatenated codewords), the one extra
+ * scalar of BlockQuant's target-aware rescale (Block Sphere VQ notes, key design 3).
+ *   rho  [n] fp16 bits (output, 2-byte aligned), round to nearest even; 1 for a zero vector.
+ * Everything else as fq_encode (same records and norms).  Runs the one-warp-per-vector kernel.
+ */
+fq_status fq_encode_rho(const void* x, fq_dtype x_type, int64_t n, int d, int k, int N,
+                        const float* rot, const float* codebook, uint8_t* codes,
+                        uint16_t* norms, uint16_t* rho, const void* search_index, void* stream);
+
+/*
+ * fq_decode_rescaled - the decoder with the rescale of Block Sphere VQ key design 3:
+ *   y_t = nu_t S_t (Pi^T zbar_t)[0:d],  S_t from `rule` (fq_rescale_rule) and the stored rho_t:
+ *   FQ_RESCALE_MSE S = rho / |zbar|^2, FQ_RESCALE_UNBIASED S = 1 / rho, FQ_RESCALE_PLAIN S = 1.
+ *   rho  [n] fp16 bits as written by fq_encode_rho.  Everything else as fq_decode.
+ */
+fq_status fq_decode_rescaled(const uint8_t* codes, const uint16_t* norms, const uint16_t* rho,
+                             int64_t n, int d, int k, int N, const float* rot,
+                             const float* codebook, int rule, void* y, fq_dtype y_type,
+                             void* stream);
+
+/*
+ * fq_encode_prod / fq_decode_prod - TurboQuant_prod (TurboQuant notes sec. 3.2), the unbiased
+ * inner-product quantizer that FibQuant is compared with: a scalar (k = 1) MSE code of the
+ * rotated unit vector at b - 1 bits per coordinate, plus the 1-bit QJL sketch (sec. 2.2) of its
+ * residual and the residual's norm.
+ *   encode: nu = |x|, u = x / nu, y = rot u, idx_r = nearest level of c1 to y_r (lowest index on
+ *           ties), r = u - rot^T c1[idx], gamma = |r|, q = sign(qjl r) with sign(0) = +1.
+ *   decode: y = nu (rot^T c1[idx] + gamma sqrt(pi/2) / d qjl^T q).
+ *   N1        levels of the scalar codebook c1 ([N1] fp32, a power of two in [2, 256]).
+ *   rot, qjl  [d, d] fp32: the Haar rotation and the QJL matrix (iid N(0,1) entries).
+ *   codes     [n, P1] bytes, P1 = fq_payload_bytes(d, 1, N1): index r at bits [r B1, (r+1) B1).
+ *   signs     [n, ceil(d / 8)] bytes: bit r % 8 of byte r / 8 is set when q_r = +1.
+ *   norms, gamma  [n] fp16 bits each (round to nearest even).
+ * Runs one warp per vector; d <= 256.
+ */
+fq_status fq_encode_prod(const void* x, fq_dtype x_type, int64_t n, int d, int N1,
+                         const float* rot, const float* c1, const float* qjl, uint8_t* codes,
+                         uint8_t* signs, uint16_t* norms, uint16_t* gamma, void* stream);
+fq_status fq_decode_prod(const uint8_t* codes, const uint8_t* signs, const uint16_t* norms,
+                         const uint16_t* gamma, int64_t n, int d, int N1, const float* rot,
+                         const float* c1, const float* qjl, void* y, fq_dtype y_type,
+                         void* stream);
+
+/*
  * Workspace bytes fq_attn_decode needs for these sizes (the split-softmax partials), or 0
  * when the sizes are unsupported.  The value depends only on the arguments.
  */
@@ -131,6 +201,45 @@ fq_status fq_attn_decode(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, i
                          const float* rotV, const float* cbV,
                          float scale, float* out, void* workspace, size_t workspace_bytes,
                          void* stream);
+
+/*
+ * fq_attn_decode_lengths - fq_attn_decode over caches of capacity T whose sequences have their
+ * own context lengths (summary sec. 1: a sequence may end anywhere; records past its end are
+ * never read and may hold anything).
+ *   lengths  [B] int32 device array, 4-byte aligned: sequence b attends over its first
+ *            clamp(lengths[b], 0, T) tokens; a sequence of length 0 outputs zeros.
+ *   Everything else as fq_attn_decode (layouts [B, Hkv, T, P]; workspace of
+ *   fq_attn_workspace_bytes(B, Hq, Hkv, T, d, kV) bytes).
+ */
+fq_status fq_attn_decode_lengths(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int d,
+                                 const int32_t* lengths, const uint8_t* k_codes,
+                                 const uint16_t* k_norms, int kK, int NK, const float* rotK,
+                                 const float* cbK, const uint8_t* v_codes,
+                                 const uint16_t* v_norms, int kV, int NV, const float* rotV,
+                                 const float* cbV, float scale, float* out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * fq_attn_decode_append - one decode step that writes its own token: the write path of the
+ * cache fused into the attention step.
+ *   k_new, v_new  [B, Hkv, d] fp16 bits: the step's key and value.  Each is encoded (brute-force
+ *                 search, as fq_encode) into record slot lengths[b] of its sequence in
+ *                 k_codes/k_norms and v_codes/v_norms ([B, Hkv, T, P] planes, written in place).
+ *   lengths       [B] int32 device array, in/out: tokens already in each sequence.  The step
+ *                 attends over lengths[b] + 1 tokens (the cache plus the new token) and, when it
+ *                 completes, adds one to lengths[b].  A sequence already holding T tokens is
+ *                 not written and not advanced (it attends over its T tokens).
+ *   Everything else as fq_attn_decode.  T must be at least 1.
+ * Enqueued as: encode of the new keys, encode of the new values, attention, combine (which
+ * advances lengths after every read of it).
+ */
+fq_status fq_attn_decode_append(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                                int B, int Hq, int Hkv, int64_t T, int d, int32_t* lengths,
+                                uint8_t* k_codes, uint16_t* k_norms, int kK, int NK,
+                                const float* rotK, const float* cbK, uint8_t* v_codes,
+                                uint16_t* v_norms, int kV, int NV, const float* rotV,
+                                const float* cbV, float scale, float* out, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /* Size of the fixed device scratch used by fq_attn_decode_noalloc (4 MiB per GPU). */
 #define FQ_ATTN_NOALLOC_SCRATCH_BYTES (4u << 20)
@@ -197,6 +306,12 @@ fq_status fq_selftest_wait_timeout(uint32_t polls, void* stream);
  *   kind           FQ_INDEX_EXACT: every codeword that can be nearest to some point of the
  *                  cell is listed (so the search equals brute force); c is ignored.
  *                  FQ_INDEX_TOPC: the c codewords nearest to each cell centre (approximate).
+ *                  FQ_INDEX_TENSOR: no grid (L and c are ignored); the codebook laid out as
+ *                  tensor-core operand tiles for half- and full-vector codes (k a multiple of
+ *                  16, at most 64; N at least 256 for k <= 32, 128 otherwise).  fq_encode then
+ *                  searches all N codewords on the tensor cores (d = 64 with k = 32 or 64,
+ *                  d = 128 with k = 64; other shapes ignore it) and returns the brute-force
+ *                  result (up to near ties of ~2^-20).  The device copy must be 16-byte aligned.
  *   L              cells per axis (2..256; L^k <= 2^22).
  *   index_host     host output buffer of index_capacity bytes, or NULL to query the size.
  *   index_bytes    (host, out) the exact size the index needs.

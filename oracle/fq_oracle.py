@@ -108,9 +108,11 @@ def block_r2_law(d: int, k: int) -> tuple[float, float]:
 
 
 def sample_source_blocks(M: int, d: int, k: int, rng: np.random.Generator) -> np.ndarray:
-    """M iid draws from f_{d,k}: radius^2 ~ Beta(k/2,(d-k)/2) times a uniform direction."""
+    """M iid draws from f_{d,k}: radius^2 ~ Beta(k/2,(d-k)/2) times a uniform direction.  For
+    the full-vector block (k = d) the block is the whole unit vector: radius 1, uniform on the
+    sphere (the Beta law degenerates at b = 0)."""
     a, b = block_r2_law(d, k)
-    r = np.sqrt(rng.beta(a, b, size=M))
+    r = np.sqrt(rng.beta(a, b, size=M)) if k < d else np.ones(M)
     u = rng.standard_normal((M, k))
     u /= np.linalg.norm(u, axis=1, keepdims=True)
     return u * r[:, None]
@@ -137,7 +139,11 @@ def quantile_levels(N: int) -> np.ndarray:
 
 
 def init_radii(d: int, k: int, N: int) -> np.ndarray:
-    """Companded Beta-quantile radii, increasing in n (general path: inverse incomplete beta)."""
+    """Companded Beta-quantile radii, increasing in n (general path: inverse incomplete beta).
+    Full-vector codes (k = d) put every codeword on the unit sphere: the block is the whole unit
+    vector, so all bits go to the angular packing ([FQ] sec. 4.2 on full-vector codes)."""
+    if k >= d:
+        return np.ones(N)
     a, b = companded_r2_law(d, k)
     return np.sqrt(special.betaincinv(a, b, quantile_levels(N)))
 
@@ -272,9 +278,22 @@ def product_codebook(c1: np.ndarray, k: int) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 
 def assign_exact(samples: np.ndarray, C: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
-    """Exact nearest codeword (k-d tree; ties have probability zero on continuous samples)."""
-    dist, idx = cKDTree(C).query(samples, k=1, workers=-1)
-    return idx.astype(np.int64), dist * dist
+    """Exact nearest codeword (ties have probability zero on continuous samples).  A k-d tree
+    for small blocks; for blocks of more than 8 coordinates (where a tree prunes nothing) plain
+    brute force by chunked matrix products, argmin of |c|^2 - 2 s.c, then the direct-form
+    squared distance of the chosen codeword."""
+    C = np.asarray(C, dtype=np.float64)
+    if C.shape[1] <= 8:
+        dist, idx = cKDTree(C).query(samples, k=1, workers=-1)
+        return idx.astype(np.int64), dist * dist
+    cc = np.sum(C * C, axis=1)
+    idx = np.empty(samples.shape[0], dtype=np.int64)
+    step = max(1, (1 << 25) // C.shape[0])
+    for s0 in range(0, samples.shape[0], step):
+        blk = samples[s0:s0 + step]
+        idx[s0:s0 + step] = np.argmin(cc[None, :] - 2.0 * (blk @ C.T), axis=1)
+    d2 = np.sum((samples - C[idx]) ** 2, axis=1)
+    return idx, d2
 
 
 def lloyd(C0: np.ndarray, samples: np.ndarray, max_iter: int = 300, tol: float = 1e-7):
@@ -398,6 +417,7 @@ def rotate_unit(x: np.ndarray, rot: np.ndarray, k: int) -> tuple[np.ndarray, np.
 def nearest_codeword(zb: np.ndarray, C: np.ndarray, chunk: int = 1 << 16):
     """Brute force over all N codewords: (argmin, gap) for blocks zb [.., k]."""
     C = np.asarray(C, dtype=np.float64)
+    chunk = max(1, min(chunk, (1 << 24) // (C.shape[0] * C.shape[1])))  # bounded temporaries
     flat = zb.reshape(-1, C.shape[1])
     idx = np.empty(flat.shape[0], dtype=np.int64)
     gap = np.empty(flat.shape[0])

@@ -25,7 +25,9 @@ OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
                    "random_access_kv_fq_b200", "tables")
 
 ROTATIONS = [(64, 17), (64, 18), (66, 17), (66, 18), (128, 17), (128, 18)]
-# (d', k, N, restarts, max_iter): large codebooks get fewer restarts / iterations (cost).
+# (d', k, N, restarts, max_iter[, training draws]): large codebooks get fewer restarts and
+# iterations (cost).  The half- and full-vector codes at N = 2^15 (the extreme-compression end of
+# the frontier) train on 4N draws for 20 iterations from the deterministic start only.
 CODEBOOKS = [
     (64, 2, 16, 8, 300),
     (64, 2, 8, 8, 300),
@@ -33,6 +35,8 @@ CODEBOOKS = [
     (66, 3, 64, 8, 300),
     (64, 4, 8, 8, 300),
     (128, 4, 4096, 2, 100),
+    (64, 32, 32768, 1, 20, 4 * 32768),
+    (64, 64, 32768, 1, 20, 4 * 32768),
 ]
 CODEBOOK_SEED = 101
 
@@ -62,13 +66,13 @@ def main(argv=None):
                           "orth_err_f32": float(np.abs(R.astype(np.float64) @ R.T.astype(np.float64)
                                                        - np.eye(dp)).max())}
         print(name, manifest[name], flush=True)
-    for dp, k, N, restarts, max_iter in CODEBOOKS:
+    for dp, k, N, restarts, max_iter, *draws in CODEBOOKS:
         name = cb_name(dp, k, N)
         if args.only is not None and name not in args.only:
             continue
         t0 = time.time()
         C, info = fo.build_codebook(dp, k, N, seed=CODEBOOK_SEED, restarts=restarts,
-                                    max_iter=max_iter)
+                                    max_iter=max_iter, M=draws[0] if draws else None)
         np.save(os.path.join(OUT, name + ".npy"), C.astype(np.float32))
         manifest[name] = {"kind": "codebook", "dp": dp, "k": k, "N": N, "seed": CODEBOOK_SEED,
                           "restarts": restarts, "max_iter": max_iter, "train_samples": info.M,

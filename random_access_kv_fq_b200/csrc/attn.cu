@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnArgs a) {
   const int tid = threadIdx.x;
   const int64_t t_begin = (int64_t)split * a.tokens_per_split;
   int64_t t_end = t_begin + a.tokens_per_split;
-  if (t_end > a.T) t_end = a.T;
+  const int64_t len_b = attn_seq_len(a, b);  // a split past the sequence's end stays empty
+  if (t_end > len_b) t_end = len_b;
 
   // rotate the group's queries once: q~_h = Pi_K pad(q_h)
   for (int e = tid; e < G * ks.dp; e += kThreads) {
@@ -217,7 +218,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AttnArgs a) {
     }
   }
   __syncthreads();
-  const float mx = red[0], inv_l = 1.f / red[1];
+  // an empty sequence (every split empty: l = 0) attends to nothing and outputs zero
+  const float mx = red[0], inv_l = red[1] > 0.f ? 1.f / red[1] : 0.f;
   for (int r = threadIdx.x; r < dpv; r += blockDim.x) {
     float v = 0.f;
     for (int s = 0; s < a.splits; ++s) {
@@ -231,6 +233,11 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AttnArgs a) {
     float v = 0.f;
     for (int r = 0; r < dpv; ++r) v = fmaf(__ldg(a.rotV + (size_t)r * dpv + c), accr[r], v);
     a.out[((size_t)b * a.Hq + h) * a.d + c] = v;
+  }
+  // the step that appended its own token advances its sequence (after every read of lengths)
+  if (a.lengths_out != nullptr && h == 0 && threadIdx.x == 0) {
+    const int32_t L = a.lengths_out[b];
+    if (L >= 0 && L < a.T) a.lengths_out[b] = L + 1;
   }
 }
 

@@ -215,8 +215,9 @@ __global__ void __launch_bounds__(kThr, Cfg<G, KB, KV, VB>::MIN_CTAS)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int64_t t_begin = (int64_t)split * a.tokens_per_split;
-  const int64_t t_end = (t_begin + a.tokens_per_split < a.T) ? t_begin + a.tokens_per_split : a.T;
-  const int n_tiles = (int)((t_end - t_begin + kT - 1) / kT);
+  const int64_t len_b = attn_seq_len(a, b);  // a split past the sequence's end stays empty
+  const int64_t t_end = (t_begin + a.tokens_per_split < len_b) ? t_begin + a.tokens_per_split : len_b;
+  const int n_tiles = t_end > t_begin ? (int)((t_end - t_begin + kT - 1) / kT) : 0;
   const size_t kv_base = ((size_t)b * a.Hkv + g) * (size_t)a.T;
 
   // sources of tile i: key records, value records, key norms, value norms
@@ -618,7 +619,8 @@ __global__ void __launch_bounds__(kThr, Cfg<G, KB, KV, VB>::MIN_CTAS)
   __syncwarp();
 
   // ---- partials of this split: (m, l, acc[d'_V]) per head, acc scaled back by sigma
-  if (!failed && !ptx::mbar_wait(bar_v, (uint32_t)(n_tiles - 1) & 1u)) failed = true;
+  if (!failed && n_tiles > 0 && !ptx::mbar_wait(bar_v, (uint32_t)(n_tiles - 1) & 1u))
+    failed = true;
   ptx::tc_fence_after();
   __syncthreads();
   float* sComb = reinterpret_cast<float*>(sAV);  // [64 coords][16 heads]: lo-row products
@@ -626,6 +628,10 @@ __global__ void __launch_bounds__(kThr, Cfg<G, KB, KV, VB>::MIN_CTAS)
   uint32_t dv[C::NVM];
   ptx::tmem_ld_cols<0, C::NVM>(tmem + lane_base + C::C_DV, dv);  // [w_hi heads | w_lo heads]
   ptx::tmem_wait_ld();
+  if (n_tiles == 0) {  // an empty split (past its sequence's end): m = -inf, l = 0, acc = 0
+#pragma unroll
+    for (int q = 0; q < C::NVM; ++q) dv[q] = 0u;
+  }
   if (tid >= 64) {  // zhat_lo rows: only the w_hi product matters at this precision
 #pragma unroll
     for (int h = 0; h < G; ++h) sComb[(tid - 64) * 16 + h] = __uint_as_float(dv[h]);

@@ -80,12 +80,24 @@ __device__ __forceinline__ bool index_matches(const uint8_t* index, int k, int N
          h->dp == dp;
 }
 
+// Record slot of input row v: v itself, or (append mode) slot lengths[b] of sequence b's
+// [T]-record plane for row v = b * hkv + g; -1 when that slot is outside the plane (the row is
+// then not written).
+__device__ __forceinline__ int64_t dest_row(const AppendMap& map, int64_t v) {
+  if (map.lengths == nullptr) return v;
+  const int64_t b = v / map.hkv;
+  const int64_t len = map.lengths[b];
+  if (len < 0 || len >= map.T) return -1;
+  return v * map.T + len;
+}
+
 template <typename TX>
 __global__ void __launch_bounds__(kWarps * 32)
     encode_generic_kernel(const TX* __restrict__ x, int64_t n, Shape s,
                           const float* __restrict__ rot, const float* __restrict__ cb,
                           uint8_t* __restrict__ codes, uint16_t* __restrict__ norms,
-                          const uint8_t* __restrict__ index) {
+                          const uint8_t* __restrict__ index, AppendMap map,
+                          uint16_t* __restrict__ rho_out) {
   extern __shared__ float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* zs = smem + warp * (s.dp + s.m);
@@ -128,7 +140,23 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     __syncwarp();
     // a5: pack, one byte per lane step; bit i of the record is bit (i % B) of index i / B
-    uint8_t* rec = codes + v * s.P;
+    // Block Sphere VQ key design 3: rho = <z, zbar>, the alignment of the unit rotated vector
+    // with its reconstruction (stored as fp16 like the norm; 1 for a zero vector)
+    if (rho_out != nullptr) {
+      float part = 0.f;
+      for (int e = lane; e < s.dp; e += 32) {
+        const int j = e / s.k;
+        part = fmaf(zs[e], __ldg(cb + (size_t)ids[j] * s.k + (e - j * s.k)), part);
+      }
+      part = warp_sum(part);
+      if (lane == 0) rho_out[v] = f32_to_f16_bits(nu > 0.f ? part : 1.f);
+    }
+    const int64_t dst = dest_row(map, v);
+    if (dst < 0) {
+      __syncwarp();
+      continue;
+    }
+    uint8_t* rec = codes + dst * s.P;
     for (int b = lane; b < s.P; b += 32) {
       uint32_t byte = 0;
       for (int t = 0; t < 8; ++t) {
@@ -138,7 +166,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       }
       rec[b] = (uint8_t)byte;
     }
-    if (lane == 0) norms[v] = f32_to_f16_bits(nu);
+    if (lane == 0) norms[dst] = f32_to_f16_bits(nu);
     __syncwarp();
   }
 }
@@ -158,20 +186,40 @@ template <typename TY>
 __global__ void __launch_bounds__(kWarps * 32)
     decode_generic_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ norms,
                           int64_t n, Shape s, const float* __restrict__ rot,
-                          const float* __restrict__ cb, TY* __restrict__ y) {
+                          const float* __restrict__ cb, TY* __restrict__ y, Gather gather,
+                          Rescale rs) {
   extern __shared__ float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* zs = smem + warp * s.dp;
   for (int64_t v = (int64_t)blockIdx.x * kWarps + warp; v < n; v += (int64_t)gridDim.x * kWarps) {
-    const uint8_t* rec = codes + v * s.P;
+    // gather mode: output row v decodes record ids[v]; an id outside the plane gives NaN
+    const int64_t src = gather.ids ? gather.ids[v] : v;
+    if (src < 0 || (gather.ids && src >= gather.n_records)) {
+#pragma unroll
+      for (int i = 0; i < kMaxD / 32; ++i) {
+        int c = lane + 32 * i;
+        if (c < s.d) store_out(y, v * s.d + c, __int_as_float(0x7fc00000));
+      }
+      continue;
+    }
+    const uint8_t* rec = codes + src * s.P;
     // a6 + a7: unpack each index and gather its codeword into the concatenated zhat
     for (int j = lane; j < s.m; j += 32) {
       int c = record_index(rec, j, s.B);
       for (int r = 0; r < s.k; ++r) zs[j * s.k + r] = __ldg(cb + (size_t)c * s.k + r);
     }
     __syncwarp();
-    // a8: y = nu (Pi^T zhat)[0:d]
-    const float nu = f16_bits_to_f32(norms[v]);
+    // a8: y = nu (Pi^T zhat)[0:d], times S of Block Sphere VQ key design 3 when rescaling
+    float nu = f16_bits_to_f32(norms[src]);
+    if (rs.rho != nullptr) {
+      const float rho = f16_bits_to_f32(rs.rho[src]);
+      float zz = 0.f;
+      for (int e = lane; e < s.dp; e += 32) zz = fmaf(zs[e], zs[e], zz);
+      zz = warp_sum(zz);
+      const float S = rs.rule == FQ_RESCALE_MSE ? rho / zz
+                      : rs.rule == FQ_RESCALE_UNBIASED ? 1.f / rho : 1.f;
+      nu *= S;
+    }
     float acc[kMaxD / 32];
 #pragma unroll
     for (int i = 0; i < kMaxD / 32; ++i) acc[i] = 0.f;
@@ -206,30 +254,32 @@ int generic_grid(int64_t n) {
 
 cudaError_t launch_encode_generic(const void* x, fq_dtype xt, int64_t n, const Shape& s,
                                   const float* rot, const float* cb, uint8_t* codes,
-                                  uint16_t* norms, const void* index, cudaStream_t st) {
+                                  uint16_t* norms, const void* index, cudaStream_t st,
+                                  AppendMap map, uint16_t* rho) {
   size_t smem = (size_t)kWarps * (s.dp + s.m) * sizeof(float);
   int grid = generic_grid(n);
   const uint8_t* ix = static_cast<const uint8_t*>(index);
   if (xt == FQ_F16)
     encode_generic_kernel<__half><<<grid, kWarps * 32, smem, st>>>(
-        static_cast<const __half*>(x), n, s, rot, cb, codes, norms, ix);
+        static_cast<const __half*>(x), n, s, rot, cb, codes, norms, ix, map, rho);
   else
     encode_generic_kernel<float><<<grid, kWarps * 32, smem, st>>>(
-        static_cast<const float*>(x), n, s, rot, cb, codes, norms, ix);
+        static_cast<const float*>(x), n, s, rot, cb, codes, norms, ix, map, rho);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_generic(const uint8_t* codes, const uint16_t* norms, int64_t n,
                                   const Shape& s, const float* rot, const float* cb, void* y,
-                                  fq_dtype yt, cudaStream_t st) {
+                                  fq_dtype yt, cudaStream_t st, Gather gather, Rescale rs) {
   size_t smem = (size_t)kWarps * s.dp * sizeof(float);
   int grid = generic_grid(n);
   if (yt == FQ_F16)
     decode_generic_kernel<__half><<<grid, kWarps * 32, smem, st>>>(codes, norms, n, s, rot, cb,
-                                                                   static_cast<__half*>(y));
+                                                                   static_cast<__half*>(y), gather, rs);
   else
     decode_generic_kernel<float><<<grid, kWarps * 32, smem, st>>>(codes, norms, n, s, rot, cb,
-                                                                  static_cast<float*>(y));
+                                                                  static_cast<float*>(y), gather,
+                                                                  rs);
   return cudaGetLastError();
 }
 

@@ -29,12 +29,20 @@ cudaError_t launch_encode_grid(const void* x, int64_t n, const float* rot, const
                                const void* index, uint8_t* codes, uint16_t* norms,
                                cudaStream_t st);
 
+// Half- and full-vector codes (d = 64 with k = 32 or 64, d = 128 with k = 64) with an
+// FQ_INDEX_TENSOR index: tensor-core GEMM search with exact re-scoring (encode_highk_sm100.cu).
+bool highk_supported(fq_dtype xt, const Shape& s, const void* x, const void* index);
+cudaError_t launch_encode_highk(const void* x, int64_t n, const Shape& s, const float* rot,
+                                const float* cb, const void* index, uint8_t* codes,
+                                uint16_t* norms, cudaStream_t st);
+
 // d = 128, k = 4, N <= 4096: tensor-core inverse rotation (decode_large_sm100.cu).
 bool decode_large_supported(fq_dtype yt, const Shape& s, const void* codes, const void* norms,
                             const void* y, const float* cb);
 cudaError_t launch_decode_large(const uint8_t* codes, const uint16_t* norms, int64_t n,
                                 const Shape& s, const float* rot, const float* cb, void* y,
-                                fq_dtype yt, cudaStream_t st);
+                                fq_dtype yt, cudaStream_t st,
+                                Gather gather = Gather{nullptr, 0});
 
 bool decode_supported(fq_dtype yt, const Shape& s, const void* codes, const void* norms,
                       const void* y);

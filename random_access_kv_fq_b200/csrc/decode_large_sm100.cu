@@ -54,6 +54,7 @@ struct DLArgs {
   const float* rot;
   const float* cb;
   void* y;
+  Gather gather;  // output row r decodes record gather.ids[r] (ids == nullptr: record r)
 };
 
 __device__ __forceinline__ uint32_t h2u_dl(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
@@ -164,11 +165,21 @@ __global__ void __launch_bounds__(kThreadsDL, 1) decode_large_kernel(DLArgs p) {
 
   auto load_rec = [&](int i, uint32_t (&w)[C::NW], float& nu) {
     const int64_t row = (first + (int64_t)i * stride) * kRowsDL + lt;
+    int64_t rec = row;
+    if (p.gather.ids != nullptr && row < p.n) {
+      rec = __ldg(p.gather.ids + row);
+      if (rec < 0 || rec >= p.gather.n_records) {  // outside the plane: a NaN row, no read
+#pragma unroll
+        for (int q = 0; q < C::NW; ++q) w[q] = 0u;
+        nu = __int_as_float(0x7fc00000);
+        return;
+      }
+    }
     if (row < p.n) {
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(p.codes + row * C::P);
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(p.codes + rec * C::P);
 #pragma unroll
       for (int q = 0; q < B; ++q) w[q] = __ldg(src + q);
-      nu = f16_bits_to_f32(__ldg(p.norms + row));
+      nu = f16_bits_to_f32(__ldg(p.norms + rec));
     } else {
 #pragma unroll
       for (int q = 0; q < B; ++q) w[q] = 0u;
@@ -330,8 +341,8 @@ bool decode_large_supported(fq_dtype yt, const Shape& s, const void* codes, cons
 
 cudaError_t launch_decode_large(const uint8_t* codes, const uint16_t* norms, int64_t n,
                                 const Shape& s, const float* rot, const float* cb, void* y,
-                                fq_dtype yt, cudaStream_t st) {
-  DLArgs p{n, codes, norms, rot, cb, y};
+                                fq_dtype yt, cudaStream_t st, Gather gather) {
+  DLArgs p{n, codes, norms, rot, cb, y, gather};
   const bool f16 = yt == FQ_F16;
   switch (s.B) {
 #define FQ_DL_CASE(BB) \

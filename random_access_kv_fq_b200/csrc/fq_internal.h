@@ -11,7 +11,7 @@
 namespace fq {
 
 constexpr int kMaxD = 256;
-constexpr int kMaxK = 8;
+constexpr int kMaxK = 256;
 constexpr int kMaxN = 65536;
 
 struct Shape {
@@ -60,6 +60,13 @@ static_assert(sizeof(IndexHeader) == 64, "index header is 64 bytes");
 constexpr uint32_t kIndexMagic = 0x58495146u;  // "FQIX"
 constexpr uint32_t kIndexVersion = 2;
 constexpr uint32_t kNoOverflow = 0xFFFFFFFFu;
+// FQ_INDEX_TENSOR buffers: the header, then (from this byte offset) N / slots chunks of
+// entry_bytes bytes, each holding `slots` codeword rows of id_bytes (= 3k + 16) fp16 elements
+// in the tensor cores' no-swizzle K-major layout (8-row x 16-byte core matrices, 128 bytes
+// apart along K, 16 * (3k + 16) bytes apart along the rows); row n of the codebook holds
+// [a_hi(k) | a_lo(k) | a_hi(k) | cc_hi | cc_lo | 0 x 14] with a = -2 c_n, cc = |c_n|^2 and
+// x_lo = fp16(x - x_hi).
+constexpr uint32_t kTensorIndexDataOffset = 128;
 
 __host__ __device__ inline bool index_has_overflow(const IndexHeader& h) {
   return h.kind == FQ_INDEX_EXACT && h.max_candidates > h.slots;
@@ -68,13 +75,50 @@ __host__ __device__ inline int index_entry_id(const uint8_t* entry, int i, int i
   return id_bytes == 1 ? entry[i] : reinterpret_cast<const uint16_t*>(entry)[i];
 }
 
+// ---- random access ---------------------------------------------------------------------------
+// Gather mode of a decode: output row v decodes record ids[v] of a plane of n_records records
+// (ids == nullptr: record v).  Ids outside [0, n_records) decode as NaN rows.
+struct Gather {
+  const int64_t* ids;
+  int64_t n_records;
+};
+// Append mode of an encode: input row v = b * hkv + g is written to record slot
+// (b * hkv + g) * T + lengths[b] of a [B, hkv, T] plane (lengths == nullptr: record v).  A slot
+// outside [0, T) is not written.
+struct AppendMap {
+  const int32_t* lengths;
+  int hkv;
+  int64_t T;
+};
+
+// Target-aware rescale of a decode (Block Sphere VQ key design 3): y = nu S (Pi^T zbar)[0:d] with
+// S from the stored rho (fp16 plane) and the rule (rho == nullptr: S = 1).
+struct Rescale {
+  const uint16_t* rho;
+  int rule;  // fq_rescale_rule
+};
+
 // ---- launchers (return cudaGetLastError() of the launch) ----------------------------------
 cudaError_t launch_encode_generic(const void* x, fq_dtype xt, int64_t n, const Shape& s,
                                   const float* rot, const float* cb, uint8_t* codes,
-                                  uint16_t* norms, const void* index, cudaStream_t st);
+                                  uint16_t* norms, const void* index, cudaStream_t st,
+                                  AppendMap map = AppendMap{nullptr, 1, 0},
+                                  uint16_t* rho = nullptr);
 cudaError_t launch_decode_generic(const uint8_t* codes, const uint16_t* norms, int64_t n,
                                   const Shape& s, const float* rot, const float* cb, void* y,
-                                  fq_dtype yt, cudaStream_t st);
+                                  fq_dtype yt, cudaStream_t st,
+                                  Gather gather = Gather{nullptr, 0},
+                                  Rescale rs = Rescale{nullptr, 0});
+
+// TurboQuant_prod (variants.cu)
+cudaError_t launch_encode_prod(const void* x, fq_dtype xt, int64_t n, int d, int N1, int B1,
+                               int P1, const float* rot, const float* c1, const float* qjl,
+                               uint8_t* codes, uint8_t* signs, uint16_t* norms, uint16_t* gamma,
+                               cudaStream_t st);
+cudaError_t launch_decode_prod(const uint8_t* codes, const uint8_t* signs, const uint16_t* norms,
+                               const uint16_t* gamma, int64_t n, int d, int N1, int B1, int P1,
+                               const float* rot, const float* c1, const float* qjl, void* y,
+                               fq_dtype yt, cudaStream_t st);
 
 struct AttnArgs {
   const uint16_t* q;
@@ -96,7 +140,21 @@ struct AttnArgs {
   float* partials;  // [B, Hq, splits, dpV + 2]
   int splits;
   int64_t tokens_per_split;
+  // per-sequence context lengths (device, [B]; nullptr: every sequence has T tokens).  Sequence
+  // b attends over its first clamp(lengths[b] + length_bias, 0, T) tokens.
+  const int32_t* lengths;
+  int length_bias;
+  // when non-null, the combine kernel adds one to lengths[b] (capped at T) after reading the
+  // partials: the decode step that appended its own token advances its sequence
+  int32_t* lengths_out;
 };
+
+// Tokens of sequence b that an attention step reads.
+__host__ __device__ inline int64_t attn_seq_len(const AttnArgs& a, int b) {
+  if (a.lengths == nullptr) return a.T;
+  int64_t L = (int64_t)a.lengths[b] + a.length_bias;
+  return L < 0 ? 0 : (L > a.T ? a.T : L);
+}
 // Validates the arguments of fq_attn_decode (everything but the workspace) and fills `a` and
 // the workspace bytes the call needs; nothing is enqueued.  T = 0 returns FQ_OK with *need = 0.
 fq_status attn_prepare(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int d,
@@ -133,6 +191,7 @@ cudaError_t wait_timeouts_decode(bool clear, unsigned* count);        // decode_
 cudaError_t wait_timeouts_decode_large(bool clear, unsigned* count);  // decode_large_sm100.cu
 cudaError_t wait_timeouts_attn(bool clear, unsigned* count);          // attn_sm100.cu
 cudaError_t wait_timeouts_selftest(bool clear, unsigned* count);      // selftest.cu
+cudaError_t wait_timeouts_encode_highk(bool clear, unsigned* count);  // encode_highk_sm100.cu
 cudaError_t launch_selftest_wait(uint32_t polls, cudaStream_t st);     // selftest.cu
 
 // sm_100a tensor-core attention (attn_sm100.cu) for the shapes it supports.

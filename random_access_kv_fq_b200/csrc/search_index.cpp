@@ -21,10 +21,75 @@
 #include <thread>
 #include <vector>
 
+#include <cuda_fp16.h>
+
 #include "fq_internal.h"
 
 namespace fq {
 namespace {
+
+uint16_t half_bits(float v) {
+  const __half h = __float2half_rn(v);
+  uint16_t b;
+  std::memcpy(&b, &h, 2);
+  return b;
+}
+float half_value(float v) { return __half2float(__float2half_rn(v)); }
+
+// FQ_INDEX_TENSOR: the codebook as tensor-core B-operand tiles (layout: kTensorIndexDataOffset).
+fq_status build_tensor_index(const float* cb, const Shape& s, void* index_host,
+                             size_t capacity, size_t* bytes) {
+  const int k = s.k, N = s.N;
+  if (k % 16 != 0 || k > 64) return FQ_ERR_UNSUPPORTED;
+  const int ch = k <= 32 ? 256 : 128;
+  if (N < ch) return FQ_ERR_UNSUPPORTED;
+  const int kop = 3 * k + 16, sbo = kop * 16;
+  const size_t chunk_bytes = (size_t)ch * kop * 2;
+  const size_t total = kTensorIndexDataOffset + (size_t)(N / ch) * chunk_bytes;
+  *bytes = total;
+  if (!index_host || capacity < total) return FQ_ERR_WORKSPACE;
+  for (size_t i = 0; i < (size_t)N * k; ++i)
+    if (!std::isfinite(cb[i])) return FQ_ERR_INVALID_ARG;
+  uint8_t* out = static_cast<uint8_t*>(index_host);
+  std::memset(out, 0, total);
+  IndexHeader hdr;
+  std::memset(&hdr, 0, sizeof(hdr));
+  hdr.magic = kIndexMagic;
+  hdr.version = kIndexVersion;
+  hdr.kind = FQ_INDEX_TENSOR;
+  hdr.k = k;
+  hdr.N = N;
+  hdr.dp = s.dp;
+  hdr.slots = ch;
+  hdr.n_cells = N / ch;
+  hdr.entry_bytes = (int32_t)chunk_bytes;
+  hdr.cells_offset = kTensorIndexDataOffset;
+  hdr.id_bytes = (uint16_t)kop;
+  std::memcpy(out, &hdr, sizeof(hdr));
+  std::vector<float> row(kop);
+  for (int n = 0; n < N; ++n) {
+    double cc = 0;
+    for (int a = 0; a < k; ++a) cc += (double)cb[(size_t)n * k + a] * cb[(size_t)n * k + a];
+    for (int a = 0; a < k; ++a) {
+      const float av = -2.0f * cb[(size_t)n * k + a];
+      const float hi = half_value(av);
+      row[a] = hi;
+      row[k + a] = av - hi;   // rounded to fp16 below
+      row[2 * k + a] = hi;
+    }
+    const float ccf = (float)cc;
+    row[3 * k] = half_value(ccf);
+    row[3 * k + 1] = ccf - half_value(ccf);
+    for (int e = 3 * k + 2; e < kop; ++e) row[e] = 0.f;
+    uint8_t* base = out + kTensorIndexDataOffset + (size_t)(n / ch) * chunk_bytes;
+    const int r = n % ch;
+    for (int e = 0; e < kop; ++e) {
+      const uint16_t b = half_bits(row[e]);
+      std::memcpy(base + (size_t)(r / 8) * sbo + (e / 8) * 128 + (r % 8) * 16 + (e % 8) * 2, &b, 2);
+    }
+  }
+  return FQ_OK;
+}
 
 struct Grid {
   int k, N, L, dp, n_cells;
@@ -125,6 +190,8 @@ extern "C" fq_status fq_build_search_index(const float* codebook_host, int d, in
   fq_status st = make_shape(d, k, N, &s);
   if (st != FQ_OK) return st;
   if (!codebook_host || !index_bytes) return FQ_ERR_INVALID_ARG;
+  if (kind == FQ_INDEX_TENSOR)
+    return build_tensor_index(codebook_host, s, index_host, index_capacity, index_bytes);
   if (kind != FQ_INDEX_EXACT && kind != FQ_INDEX_TOPC) return FQ_ERR_INVALID_ARG;
   if (L < 2 || L > 256) return FQ_ERR_UNSUPPORTED;
   double cells_d = std::pow((double)L, k);
