@@ -31,7 +31,8 @@ cudaError_t launch_encode_grid(const void* x, int64_t n, const float* rot, const
 
 // Half- and full-vector codes (d = 64 with k = 32 or 64, d = 128 with k = 64) with an
 // FQ_INDEX_TENSOR index: tensor-core GEMM search with exact re-scoring (encode_highk_sm100.cu).
-bool highk_supported(fq_dtype xt, const Shape& s, const void* x, const void* index);
+bool highk_supported(fq_dtype xt, const Shape& s, const void* x, const void* index,
+                     const float* rot, const float* cb);
 cudaError_t launch_encode_highk(const void* x, int64_t n, const Shape& s, const float* rot,
                                 const float* cb, const void* index, uint8_t* codes,
                                 uint16_t* norms, cudaStream_t st);

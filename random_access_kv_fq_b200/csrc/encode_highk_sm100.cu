@@ -431,8 +431,11 @@ cudaError_t launch_hk(const HParams& p, cudaStream_t st) {
 
 }  // namespace
 
-bool highk_supported(fq_dtype xt, const Shape& s, const void* x, const void* index) {
+bool highk_supported(fq_dtype xt, const Shape& s, const void* x, const void* index,
+                     const float* rot, const float* cb) {
   if (xt != FQ_F16 || index == nullptr) return false;
+  if ((reinterpret_cast<uintptr_t>(rot) & 15) || (reinterpret_cast<uintptr_t>(cb) & 15))
+    return false;
   if (!((s.d == 64 && (s.k == 32 || s.k == 64)) || (s.d == 128 && s.k == 64))) return false;
   if (s.dp != s.d || s.N < (s.k <= 32 ? 256 : 128) || s.N > 65536) return false;
   if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(index) & 15))

@@ -73,7 +73,7 @@ fq_status fq_encode(const void* x, fq_dtype x_type, int64_t n, int d, int k, int
       !aligned(codebook, 4) || (search_index && !aligned(search_index, 8)))
     return FQ_ERR_ALIGNMENT;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (sm100::highk_supported(x_type, s, x, search_index))
+  if (sm100::highk_supported(x_type, s, x, search_index, rot, codebook))
     return from_cuda(sm100::launch_encode_highk(x, n, s, rot, codebook, search_index, codes,
                                                 norms, cs));
   if (sm100::encode_large_supported(x_type, s, x, codes, codebook, search_index))
