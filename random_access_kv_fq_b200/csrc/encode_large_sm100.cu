@@ -498,318 +498,6 @@ cudaError_t launch_large(const LParams& p, cudaStream_t st) {
 }
 
 
-// ---- top-c / exact grid search (Block Sphere VQ notes, key design 2) for N = 4096 ----------
-// The block's cell on an L^4 grid (host-built index) names up to 8 candidate codewords; the
-// nearest of them by the direct fp32 squared distance wins, the lower index on equality (as the
-// oracle).  Same rotation as above; the search of a tile's 32 blocks is split over the four
-// warpgroups (blocks 8 wg .. 8 wg + 7 of every row), and each writes its 96 record bits (three
-// whole words at N = 4096) straight to global memory.
-constexpr int kBG = 12;                    // index bits (N = 4096)
-constexpr int kNG = 1 << kBG;
-constexpr int kPG = kML * kBG / 8;         // 48-byte records
-
-struct GCfg {
-  static constexpr int OFF_PI = 0;                     // as LCfg: 64 KB rotation operand
-  static constexpr int OFF_TBL = 2 * 256 * 128;        // N x float4 codebook
-  static constexpr int OFF_ZERO = OFF_TBL + kNG * 16;    // [128] rows with nu = 0
-  static constexpr int OFF_BAR = OFF_ZERO + kRowsL;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
-};
-
-struct GParams {
-  int64_t n;
-  const uint16_t* x;
-  const float* rot;
-  const float* cb;
-  const uint8_t* index;
-  uint8_t* codes;
-  uint16_t* norms;
-};
-
-__device__ __forceinline__ void scan_sync() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kScanThreads) : "memory");
-}
-
-__global__ void __launch_bounds__(kThreadsL, 1) encode_grid_kernel(GParams p) {
-  using C = GCfg;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sPi = smem + C::OFF_PI;
-  const float4* sTbl = reinterpret_cast<const float4*>(smem + C::OFF_TBL);
-  uint64_t* x_ready = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // x staged (4 warps)
-  uint64_t* rot_done = x_ready + 1;                                   // rotation MMA done
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(rot_done + 1);
-  volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
-  uint8_t* sZero = smem + C::OFF_ZERO;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wg = warp >> 2;
-  const int row = 32 * (warp & 3) + lane;
-  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-  const int64_t n_tiles = (p.n + kRowsL - 1) / kRowsL;
-  const int n_local =
-      (blockIdx.x < n_tiles) ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
-
-  // ---- set-up ----
-  if (warp == 16) {
-    ptx::tmem_alloc(sTmem, 512);
-    ptx::tmem_relinquish();
-  }
-  if (tid == 0) {
-    ptx::mbar_init(x_ready, kRowsL / 32);
-    ptx::mbar_init(rot_done, 1);
-    *sAbort = 0;
-    ptx::fence_mbar_init();
-  }
-  // the index, when it describes this codebook (else exact brute force over the table)
-  const IndexHeader h = *reinterpret_cast<const IndexHeader*>(p.index);
-  const bool use_index = h.magic == kIndexMagic && h.version == kIndexVersion && h.k == 4 &&
-                         h.N == kNG && h.dp == kDL && h.id_bytes == 2 && h.slots >= 1 &&
-                         h.slots <= 8 && h.entry_bytes <= 16 && (h.entry_bytes & 3) == 0 &&
-                         !index_has_overflow(h);
-  // rotation operand (as in encode_large_kernel)
-#pragma unroll 1
-  for (int e0 = 0; e0 < kDL * kDL; e0 += 8 * kThreadsL) {
-    float v[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int e = e0 + q * kThreadsL + tid;
-      v[q] = e < kDL * kDL ? __ldg(p.rot + e) : 0.f;
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int e = e0 + q * kThreadsL + tid;
-      if (e < kDL * kDL) {
-        const int n = e >> 7, c = e & 127;
-        const __half hi = __float2half_rn(v[q]);
-        const __half lo = __float2half_rn((v[q] - __half2float(hi)) * 4096.0f);
-        uint8_t* half_tile = sPi + (c >> 6) * (256 * 128);
-        *reinterpret_cast<__half*>(half_tile + ptx::sw128_offset(n, c & 63)) = hi;
-        *reinterpret_cast<__half*>(half_tile + ptx::sw128_offset(128 + n, c & 63)) = lo;
-      }
-    }
-  }
-  // fp32 codebook table
-#pragma unroll 1
-  for (int c0 = 0; c0 < kNG; c0 += 4 * kThreadsL) {
-    float4 v[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = c0 + q * kThreadsL + tid;
-      v[q] = c < kNG ? __ldg(reinterpret_cast<const float4*>(p.cb) + c) : make_float4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = c0 + q * kThreadsL + tid;
-      if (c < kNG) const_cast<float4*>(sTbl)[c] = v[q];
-    }
-  }
-  ptx::fence_proxy_async_smem();
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-  const uint32_t tmem = *sTmem;
-  constexpr uint32_t TM_X = 256;
-
-  if (warp == 16) {
-    // ---- MMA issuer: the rotation of each tile ----
-    if (lane == 0) {
-      constexpr uint32_t idesc_rot = ptx::idesc_f16_f32(128, 256);
-      const uint32_t pi = ptx::smem_u32(sPi);
-      int issued = 0;
-      for (int i = 0; i < n_local; ++i) {
-        if (!wait_l(x_ready, (uint32_t)i & 1u, sAbort)) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          ptx::umma_f16_ts(tmem, tmem + TM_X + 8 * ks,
-                           ptx::sdesc_kmajor_sw128(pi + (ks >> 2) * (256 * 128) + (ks & 3) * 32),
-                           idesc_rot, ks > 0 ? 1u : 0u);
-        ptx::umma_commit(rot_done);
-        issued = i + 1;
-      }
-      if (issued > 0) ptx::mbar_wait(rot_done, (uint32_t)(issued - 1) & 1u);  // bounded
-    }
-    __syncwarp();
-  } else {
-    float nu = 0.f;
-    for (int i = 0; i < n_local; ++i) {
-      const int64_t tile = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
-      const int64_t vrow = tile * kRowsL + row;
-      bool fail = false;
-      scan_sync();  // the previous tile's z has been read by every warpgroup
-      if (wg == 0) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.x + vrow * kDL);
-        float part[8];
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t r16[16];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint4 v = vrow < p.n ? __ldg(src + 4 * q + e) : make_uint4(0u, 0u, 0u, 0u);
-            r16[4 * e] = v.x; r16[4 * e + 1] = v.y; r16[4 * e + 2] = v.z; r16[4 * e + 3] = v.w;
-          }
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            float a2 = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r16[8 * hh + e]));
-              a2 = fmaf(f.x, f.x, a2);
-              a2 = fmaf(f.y, f.y, a2);
-            }
-            part[2 * q + hh] = a2;
-          }
-          ptx::tmem_st16(tmem + lane_base + TM_X + 16 * q, r16);
-        }
-        nu = sqrtf(((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7])));
-        const float rinv = nu > 0.f ? __frcp_rn(nu) : 0.f;
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(x_ready);
-        bool ok = true;
-        if (lane == 0) ok = wait_l(rot_done, (uint32_t)i & 1u, sAbort);
-        fail = __shfl_sync(0xffffffffu, (int)ok, 0) == 0;
-        __syncwarp();
-        ptx::tc_fence_after();
-        if (!fail) {  // z = (D_hi + 2^-12 D_lo) / nu into columns 0..127
-#pragma unroll 1
-          for (int q = 0; q < 16; ++q) {
-            uint32_t hv[8], lv[8];
-            ptx::tmem_ld8(tmem + lane_base + 8 * q, hv);
-            ptx::tmem_ld8(tmem + lane_base + 128 + 8 * q, lv);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              hv[e] = __float_as_uint(
-                  fmaf(__uint_as_float(lv[e]), kLoScaleL * rinv, __uint_as_float(hv[e]) * rinv));
-            ptx::tmem_st8(tmem + lane_base + 8 * q, hv);
-          }
-          ptx::tmem_wait_st();
-        }
-        if (vrow < p.n) p.norms[vrow] = f32_to_f16_bits(nu);
-        sZero[row] = nu > 0.f ? 0 : 1;  // a zero vector stores index 0 in every block
-      }
-      ptx::tc_fence_before();
-      if (scan_sync_or(fail)) break;  // z is in place
-      ptx::tc_fence_after();
-      // ---- this warpgroup's blocks 8 wg .. 8 wg + 7 of this row ----
-      uint32_t zw[32];
-      ptx::tmem_ld_cols<0, 32>(tmem + lane_base + 32 * wg, zw);
-      ptx::tmem_wait_ld();
-      uint32_t rec[3] = {0u, 0u, 0u};
-      if (sZero[row]) {
-        // index 0 everywhere: rec stays zero
-      } else if (use_index) {
-#pragma unroll
-        for (int b0 = 0; b0 < 8; b0 += 4) {  // 4 blocks: cells, their entries in one batch, search
-          uint4 ent[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int b = b0 + u;
-            int flat = 0, mul = 1;
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-              const float t = (__uint_as_float(zw[4 * b + a]) - h.lo) * h.inv_h;
-              int c = (int)floorf(t);
-              c = c < 0 ? 0 : (c >= h.L ? h.L - 1 : c);
-              flat += c * mul;
-              mul *= h.L;
-            }
-            const uint8_t* e = p.index + h.cells_offset + (size_t)flat * h.entry_bytes;
-            ent[u] = h.entry_bytes == 16
-                         ? __ldg(reinterpret_cast<const uint4*>(e))
-                         : make_uint4(__ldg(reinterpret_cast<const uint32_t*>(e)),
-                                      h.entry_bytes > 4 ? __ldg(reinterpret_cast<const uint32_t*>(e) + 1) : 0u,
-                                      h.entry_bytes > 8 ? __ldg(reinterpret_cast<const uint32_t*>(e) + 2) : 0u, 0u);
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int b = b0 + u;
-            const uint32_t words[4] = {ent[u].x, ent[u].y, ent[u].z, ent[u].w};
-            float best = INFINITY;
-            int bi = 0;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              if (q < h.slots) {
-                const int c = (int)((words[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
-                const float4 cv = sTbl[c];
-                const float d0 = __uint_as_float(zw[4 * b]) - cv.x;
-                const float d1 = __uint_as_float(zw[4 * b + 1]) - cv.y;
-                const float d2 = __uint_as_float(zw[4 * b + 2]) - cv.z;
-                const float d3 = __uint_as_float(zw[4 * b + 3]) - cv.w;
-                const float dd = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
-                if (q == 0 || better(dd, c, best, bi)) {
-                  best = dd;
-                  bi = c;
-                }
-              }
-            }
-            const uint32_t ix = (uint32_t)bi & (kNG - 1);
-            const uint32_t bit = (uint32_t)(b * kBG);
-            rec[bit >> 5] |= ix << (bit & 31);
-            if ((bit & 31) + kBG > 32) rec[(bit >> 5) + 1] |= ix >> (32 - (bit & 31));
-          }
-        }
-      } else {
-#pragma unroll
-        for (int b = 0; b < 8; ++b) {  // no usable index: exact brute force over the table
-          float best = INFINITY;
-          int bi = 0;
-#pragma unroll 4
-          for (int c = 0; c < kNG; ++c) {
-            const float4 cv = sTbl[c];
-            const float d0 = __uint_as_float(zw[4 * b]) - cv.x;
-            const float d1 = __uint_as_float(zw[4 * b + 1]) - cv.y;
-            const float d2 = __uint_as_float(zw[4 * b + 2]) - cv.z;
-            const float d3 = __uint_as_float(zw[4 * b + 3]) - cv.w;
-            const float dd = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
-            if (dd < best) {
-              best = dd;
-              bi = c;
-            }
-          }
-          const uint32_t ix = (uint32_t)bi & (kNG - 1);
-          const uint32_t bit = (uint32_t)(b * kBG);
-          rec[bit >> 5] |= ix << (bit & 31);
-          if ((bit & 31) + kBG > 32) rec[(bit >> 5) + 1] |= ix >> (32 - (bit & 31));
-        }
-      }
-      ptx::tc_fence_before();
-      if (vrow < p.n) {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(p.codes + vrow * kPG) + 3 * wg;
-        dst[0] = rec[0];
-        dst[1] = rec[1];
-        dst[2] = rec[2];
-      }
-    }
-  }
-
-  ptx::tc_fence_before();
-  __syncthreads();
-  if (tid == 0 && *sAbort) atomicAdd(&g_encl_wait_timeouts, 1u);
-  if (warp == 16) {
-    ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 512);
-  }
-}
-
-cudaError_t launch_grid(const GParams& p, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(encode_grid_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, GCfg::SMEM);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (p.n + kRowsL - 1) / kRowsL;
-  const int ctas = (int)(tiles < sms ? tiles : sms);
-  encode_grid_kernel<<<ctas, kThreadsL, GCfg::SMEM, st>>>(p);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 bool encode_large_supported(fq_dtype xt, const Shape& s, const void* x, const void* codes,
@@ -823,26 +511,6 @@ bool encode_large_supported(fq_dtype xt, const Shape& s, const void* x, const vo
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   return major == 10;
-}
-
-bool encode_grid_supported(fq_dtype xt, const Shape& s, const void* x, const void* codes,
-                           const float* cb, const void* index) {
-  if (xt != FQ_F16 || s.d != kDL || s.k != 4 || s.B != kBG || index == nullptr) return false;
-  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(codes) & 3) ||
-      (reinterpret_cast<uintptr_t>(cb) & 15) || (reinterpret_cast<uintptr_t>(index) & 15))
-    return false;
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  return major == 10;
-}
-
-cudaError_t launch_encode_grid(const void* x, int64_t n, const float* rot, const float* cb,
-                               const void* index, uint8_t* codes, uint16_t* norms,
-                               cudaStream_t st) {
-  GParams p{n, static_cast<const uint16_t*>(x), rot, cb, static_cast<const uint8_t*>(index),
-            codes, norms};
-  return launch_grid(p, st);
 }
 
 cudaError_t launch_encode_large(const void* x, int64_t n, const Shape& s, const float* rot,

@@ -365,6 +365,7 @@ fq_status fq_wait_status(unsigned* timed_out, int clear) {
   unsigned n = 0;
   cudaError_t (*readers[])(bool, unsigned*) = {wait_timeouts_encode, wait_timeouts_encode_large,
                                                wait_timeouts_encode_highk,
+                                               wait_timeouts_encode_grid,
                                                wait_timeouts_decode, wait_timeouts_decode_large,
                                                wait_timeouts_attn, wait_timeouts_selftest};
   for (auto rd : readers)

@@ -192,6 +192,7 @@ cudaError_t wait_timeouts_decode_large(bool clear, unsigned* count);  // decode_
 cudaError_t wait_timeouts_attn(bool clear, unsigned* count);          // attn_sm100.cu
 cudaError_t wait_timeouts_selftest(bool clear, unsigned* count);      // selftest.cu
 cudaError_t wait_timeouts_encode_highk(bool clear, unsigned* count);  // encode_highk_sm100.cu
+cudaError_t wait_timeouts_encode_grid(bool clear, unsigned* count);   // encode_grid_sm100.cu
 cudaError_t launch_selftest_wait(uint32_t polls, cudaStream_t st);     // selftest.cu
 
 // sm_100a tensor-core attention (attn_sm100.cu) for the shapes it supports.
