@@ -89,7 +89,9 @@ __device__ __forceinline__ bool better_g(float v, int i, float bv, int bi) {
   return v < bv || (v == bv && i < bi);
 }
 
-__global__ void __maxnreg__(112)
+// 18 warps: with the register file split over four sub-partitions (five warps on two of them),
+// at most 96 registers per thread fit one CTA per SM.
+__global__ void __launch_bounds__(kThreadsG, 1)
     encode_grid_kernel(const __grid_constant__ CUtensorMap xmap, GParams p) {
   using C = GCfg;
   extern __shared__ uint8_t smem_raw[];
