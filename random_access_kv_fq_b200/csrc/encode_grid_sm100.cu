@@ -89,6 +89,44 @@ __device__ __forceinline__ bool better_g(float v, int i, float bv, int bi) {
   return v < bv || (v == bv && i < bi);
 }
 
+// Exact fp32 re-scoring of a block's candidate list (the rare case where the fixed-point
+// distances cannot separate the best two); lowest index on equal distances.  Out of line so
+// that the hot loop stays small in the instruction cache.
+__device__ __noinline__ int rerank_exact(float z0, float z1, float z2, float z3, uint4 ent,
+                                         int slots, const float4* __restrict__ cb) {
+  const uint32_t words[4] = {ent.x, ent.y, ent.z, ent.w};
+  float best = INFINITY;
+  int bi = 0x7fffffff;
+  for (int q = 0; q < slots; ++q) {
+    const int c = (int)((words[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+    const float4 cv = __ldg(cb + c);
+    const float e0 = z0 - cv.x, e1 = z1 - cv.y, e2 = z2 - cv.z, e3 = z3 - cv.w;
+    const float dd = fmaf(e0, e0, fmaf(e1, e1, fmaf(e2, e2, e3 * e3)));
+    if (better_g(dd, c, best, bi)) {
+      best = dd;
+      bi = c;
+    }
+  }
+  return bi;
+}
+
+// Exact brute force over all N codewords (an index that does not describe this codebook).
+__device__ __noinline__ int brute_exact(float z0, float z1, float z2, float z3,
+                                        const float4* __restrict__ cb) {
+  float best = INFINITY;
+  int bi = 0;
+  for (int c = 0; c < kNG; ++c) {
+    const float4 cv = __ldg(cb + c);
+    const float d0 = z0 - cv.x, d1 = z1 - cv.y, d2 = z2 - cv.z, d3 = z3 - cv.w;
+    const float dd = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
+    if (dd < best) {
+      best = dd;
+      bi = c;
+    }
+  }
+  return bi;
+}
+
 // 18 warps: with the register file split over four sub-partitions (five warps on two of them),
 // at most 96 registers per thread fit one CTA per SM.
 __global__ void __launch_bounds__(kThreadsG, 1)
@@ -285,34 +323,34 @@ __global__ void __launch_bounds__(kThreadsG, 1)
       if (lane == 0) ptx::mbar_arrive(&x_empty[s]);  // this warp no longer reads the stage
       if (fail) break;
       const float rinv = nu > 0.f ? __frcp_rn(nu) : 0.f;
-      // z of this thread's 8 blocks: (D_hi + 2^-12 D_lo) / nu
-      fail = !wait_g(&z_full[b], (uint32_t)(i >> 1) & 1u, sAbort);
-      float z[32];
-      if (!fail) {
-        ptx::tc_fence_after();
-        const uint32_t dz = tmem + lane_base + (uint32_t)(b * 256 + 32 * wg);
+      // blocks 8 wg .. 8 wg + 7 in two halves of four: z = (D_hi + 2^-12 D_lo) / nu from the
+      // accumulator, the four cells, their index entries (loaded together), the candidates
+      fail = __any_sync(0xffffffffu, !wait_g(&z_full[b], (uint32_t)(i >> 1) & 1u, sAbort));
+      if (!fail) ptx::tc_fence_after();
+      const uint32_t dz = tmem + lane_base + (uint32_t)(b * 256 + 32 * wg);
+      uint32_t rec[3] = {0u, 0u, 0u};
 #pragma unroll
-        for (int h16 = 0; h16 < 2; ++h16) {
+      for (int hb = 0; hb < 2; ++hb) {
+        float z[16];
+        if (!fail) {
           uint32_t hv[16], lv[16];
-          ptx::tmem_ld16(dz + 16 * h16, hv);
-          ptx::tmem_ld16(dz + 128 + 16 * h16, lv);
+          ptx::tmem_ld16(dz + 16 * hb, hv);
+          ptx::tmem_ld16(dz + 128 + 16 * hb, lv);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            z[16 * h16 + e] = fmaf(__uint_as_float(lv[e]), kLoScaleG * rinv,
-                                   __uint_as_float(hv[e]) * rinv);
+            z[e] = fmaf(__uint_as_float(lv[e]), kLoScaleG * rinv, __uint_as_float(hv[e]) * rinv);
         }
-        ptx::tc_fence_before();
-      }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&z_empty[b]);
-      if (fail) break;
-      uint32_t rec[3] = {0u, 0u, 0u};
-      if (nu > 0.f) {  // a zero vector keeps index 0 in every block
+        if (hb == 1) {  // the accumulator is read: the MMA of tile i + 2 may overwrite it
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&z_empty[b]);
+        }
+        if (fail || !(nu > 0.f)) continue;  // a zero vector keeps index 0 in every block
         if (use_index) {
-          uint4 ent[8];
+          uint4 ent[4];
 #pragma unroll
-          for (int bk = 0; bk < 8; ++bk) {
+          for (int bk = 0; bk < 4; ++bk) {
             int flat = 0, mul = 1;
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
@@ -330,7 +368,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                                        h.entry_bytes > 8 ? __ldg(reinterpret_cast<const uint32_t*>(e) + 2) : 0u, 0u);
           }
 #pragma unroll
-          for (int bk = 0; bk < 8; ++bk) {
+          for (int bk = 0; bk < 4; ++bk) {
             const uint32_t words[4] = {ent[bk].x, ent[bk].y, ent[bk].z, ent[bk].w};
             const float z0 = z[4 * bk] + 3.f, z1 = z[4 * bk + 1] + 3.f;
             const float z2 = z[4 * bk + 2] + 3.f, z3 = z[4 * bk + 3] + 3.f;
@@ -351,54 +389,31 @@ __global__ void __launch_bounds__(kThreadsG, 1)
               }
             }
             int bi = i1;
-            // each fixed-point distance is within (2^-14 + 2^-21) sqrt(d) + 2.4e-7 d + 1e-9 of the
-            // exact one (codeword rounding 2^-16 per coordinate, z + 3 rounding 2^-23, fp32
-            // sums): unless the best two are closer than twice that, the approximate winner
-            // is the exact winner
-            if (!(d2 - d1 > 1.25e-4f * sqrtf(d2) + 6e-7f * d2 + 1e-8f)) {
-              float best = INFINITY;
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                if (q >= h.slots) break;
-                const int c = (int)((words[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
-                const float4 cv = __ldg(reinterpret_cast<const float4*>(p.cb) + c);
-                const float e0 = z[4 * bk] - cv.x, e1 = z[4 * bk + 1] - cv.y;
-                const float e2 = z[4 * bk + 2] - cv.z, e3 = z[4 * bk + 3] - cv.w;
-                const float dd = fmaf(e0, e0, fmaf(e1, e1, fmaf(e2, e2, e3 * e3)));
-                if (q == 0 || better_g(dd, c, best, bi)) {
-                  best = dd;
-                  bi = c;
-                }
-              }
-            }
+            // each fixed-point distance is within (2^-14 + 2^-21) sqrt(d) + 2.4e-7 d + 1e-9 of
+            // the exact one (codeword rounding 2^-16 per coordinate, z + 3 rounding 2^-23, fp32
+            // sums): unless the best two are closer than twice that, the approximate winner is
+            // the exact winner
+            if (!(d2 - d1 > 1.25e-4f * sqrtf(d2) + 6e-7f * d2 + 1e-8f))
+              bi = rerank_exact(z[4 * bk], z[4 * bk + 1], z[4 * bk + 2], z[4 * bk + 3], ent[bk],
+                                h.slots, reinterpret_cast<const float4*>(p.cb));
             const uint32_t ix = (uint32_t)bi & (kNG - 1);
-            const uint32_t bit = (uint32_t)(bk * kBG);
+            const uint32_t bit = (uint32_t)((4 * hb + bk) * kBG);
             rec[bit >> 5] |= ix << (bit & 31);
             if ((bit & 31) + kBG > 32) rec[(bit >> 5) + 1] |= ix >> (32 - (bit & 31));
           }
         } else {
 #pragma unroll
-          for (int bk = 0; bk < 8; ++bk) {  // no usable index: exact brute force (fp32, L1/L2)
-            float best = INFINITY;
-            int bi = 0;
-#pragma unroll 4
-            for (int c = 0; c < kNG; ++c) {
-              const float4 cv = __ldg(reinterpret_cast<const float4*>(p.cb) + c);
-              const float d0 = z[4 * bk] - cv.x, d1 = z[4 * bk + 1] - cv.y;
-              const float d2 = z[4 * bk + 2] - cv.z, d3 = z[4 * bk + 3] - cv.w;
-              const float dd = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
-              if (dd < best) {
-                best = dd;
-                bi = c;
-              }
-            }
+          for (int bk = 0; bk < 4; ++bk) {  // no usable index: exact brute force (fp32, L1/L2)
+            const int bi = brute_exact(z[4 * bk], z[4 * bk + 1], z[4 * bk + 2], z[4 * bk + 3],
+                                       reinterpret_cast<const float4*>(p.cb));
             const uint32_t ix = (uint32_t)bi & (kNG - 1);
-            const uint32_t bit = (uint32_t)(bk * kBG);
+            const uint32_t bit = (uint32_t)((4 * hb + bk) * kBG);
             rec[bit >> 5] |= ix << (bit & 31);
             if ((bit & 31) + kBG > 32) rec[(bit >> 5) + 1] |= ix >> (32 - (bit & 31));
           }
         }
       }
+      if (fail) break;
       if (vrow < p.n) {  // this warpgroup's three record words
         uint32_t* dst = reinterpret_cast<uint32_t*>(p.codes + vrow * kPG) + 3 * wg;
         dst[0] = rec[0];
