@@ -49,13 +49,14 @@ constexpr int kXStage = kRowsG * kDG * 2;  // 32 KB: two [128 x 64] fp16 boxes
 
 __device__ unsigned int g_encg_wait_timeouts = 0;  // CTAs whose bounded waits gave up
 
-constexpr int kStagesG = 3;               // x tiles in flight
+constexpr int kStagesG = 2;               // x tiles in flight
 
 struct GCfg {
   static constexpr int OFF_PI = 0;                      // [2 K halves][256 rows x 128 B]
   static constexpr int OFF_X = OFF_PI + 2 * 256 * 128;  // [stages][2 boxes][128 x 128 B]
   static constexpr int OFF_TBL = OFF_X + kStagesG * kXStage;  // N x 4 int16 codebook
-  static constexpr int OFF_NU = OFF_TBL + kNG * 8;      // [stages][128] norms
+  static constexpr int OFF_F32 = OFF_TBL + kNG * 8;     // N x float4 codebook (exact scores)
+  static constexpr int OFF_NU = OFF_F32 + kNG * 16;     // [stages][128] norms
   static constexpr int OFF_BAR = OFF_NU + kStagesG * kRowsG * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
@@ -90,33 +91,36 @@ __device__ __forceinline__ bool better_g(float v, int i, float bv, int bi) {
 }
 
 // Exact fp32 re-scoring of a block's candidate list (the rare case where the fixed-point
-// distances cannot separate the best two); lowest index on equal distances.  Out of line so
-// that the hot loop stays small in the instruction cache.
-__device__ __noinline__ int rerank_exact(float z0, float z1, float z2, float z3, uint4 ent,
-                                         int slots, const float4* __restrict__ cb) {
+// distances cannot separate the best two); lowest index on equal distances.
+__device__ __forceinline__ int rerank_exact(float z0, float z1, float z2, float z3, uint4 ent,
+                                            int slots, const float4* tbl) {
   const uint32_t words[4] = {ent.x, ent.y, ent.z, ent.w};
   float best = INFINITY;
   int bi = 0x7fffffff;
-  for (int q = 0; q < slots; ++q) {
-    const int c = (int)((words[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
-    const float4 cv = __ldg(cb + c);
-    const float e0 = z0 - cv.x, e1 = z1 - cv.y, e2 = z2 - cv.z, e3 = z3 - cv.w;
-    const float dd = fmaf(e0, e0, fmaf(e1, e1, fmaf(e2, e2, e3 * e3)));
-    if (better_g(dd, c, best, bi)) {
-      best = dd;
-      bi = c;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    if (q < slots) {
+      const int c = (int)((words[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+      const float4 cv = tbl[c];
+      const float e0 = z0 - cv.x, e1 = z1 - cv.y, e2 = z2 - cv.z, e3 = z3 - cv.w;
+      const float dd = fmaf(e0, e0, fmaf(e1, e1, fmaf(e2, e2, e3 * e3)));
+      if (better_g(dd, c, best, bi)) {
+        best = dd;
+        bi = c;
+      }
     }
   }
   return bi;
 }
 
 // Exact brute force over all N codewords (an index that does not describe this codebook).
+// Out of line: it only runs for such an index.
 __device__ __noinline__ int brute_exact(float z0, float z1, float z2, float z3,
-                                        const float4* __restrict__ cb) {
+                                        const float4* tbl) {
   float best = INFINITY;
   int bi = 0;
   for (int c = 0; c < kNG; ++c) {
-    const float4 cv = __ldg(cb + c);
+    const float4 cv = tbl[c];
     const float d0 = z0 - cv.x, d1 = z1 - cv.y, d2 = z2 - cv.z, d3 = z3 - cv.w;
     const float dd = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
     if (dd < best) {
@@ -138,6 +142,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
   uint8_t* sPi = smem + C::OFF_PI;
   uint8_t* sX = smem + C::OFF_X;
   uint2* sTbl = reinterpret_cast<uint2*>(smem + C::OFF_TBL);
+  float4* sF32 = reinterpret_cast<float4*>(smem + C::OFF_F32);
   float* sNu = reinterpret_cast<float*>(smem + C::OFF_NU);
   uint64_t* x_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [3] x tile landed
   uint64_t* x_empty = x_full + kStagesG;  // [3] rotation done and the stage's norms read
@@ -160,8 +165,8 @@ __global__ void __launch_bounds__(kThreadsG, 1)
   if (tid == 0) {
     for (int s = 0; s < kStagesG; ++s) {
       ptx::mbar_init(&x_full[s], 1);
-      ptx::mbar_init(&x_empty[s], 1 + kSearchThreads / 32);
-      ptx::mbar_init(&nu_full[s], 4);
+      ptx::mbar_init(&x_empty[s], 2 + kSearchThreads / 32);
+      ptx::mbar_init(&nu_full[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&z_full[s], 1);
@@ -216,6 +221,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
           return (uint32_t)((int)t + 32768);
         };
         sTbl[c] = make_uint2(fx(v[q].x) | (fx(v[q].y) << 16), fx(v[q].z) | (fx(v[q].w) << 16));
+        sF32[c] = v[q];
       }
     }
   }
@@ -226,24 +232,76 @@ __global__ void __launch_bounds__(kThreadsG, 1)
   const uint32_t tmem = *sTmem;
 
   if (warp == 0) {
-    // ---- producer: x tiles into the ring of kStagesG stages ----
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < n_local; ++i) {
-        const int s = i % kStagesG;
-        if (i >= kStagesG &&
-            !wait_g(&x_empty[s], (uint32_t)((i / kStagesG) - 1) & 1u, sAbort))
-          break;
+    // ---- producer warp: x tiles into the ring (lane 0), and the norms of each landed tile
+    //      (four rows per lane, from the swizzled stage) handed to the search warps ----
+    if (lane == 0)
+      for (int i = 0; i < n_local && i < kStagesG; ++i) {
         const int64_t tile = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
-        ptx::mbar_arrive_expect_tx(&x_full[s], kXStage);
-        ptx::tma_load_2d(sX + s * kXStage, &xmap, &x_full[s], 0, (int)(tile * kRowsG));
-        ptx::tma_load_2d(sX + s * kXStage + kXStage / 2, &xmap, &x_full[s], 64,
+        ptx::mbar_arrive_expect_tx(&x_full[i], kXStage);
+        ptx::tma_load_2d(sX + i * kXStage, &xmap, &x_full[i], 0, (int)(tile * kRowsG));
+        ptx::tma_load_2d(sX + i * kXStage + kXStage / 2, &xmap, &x_full[i], 64,
                          (int)(tile * kRowsG));
-        issued = i + 1;
       }
-      for (int t = issued - kStagesG < 0 ? 0 : issued - kStagesG; t < issued; ++t)
-        ptx::mbar_wait(&x_full[t % kStagesG], (uint32_t)(t / kStagesG) & 1u);  // land first
+    int issued = n_local < kStagesG ? n_local : kStagesG;
+    for (int i = 0; i < n_local; ++i) {
+      const int s = i % kStagesG;
+      const int64_t tile = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+      if (__any_sync(0xffffffffu, !wait_g(&x_full[s], (uint32_t)(i / kStagesG) & 1u, sAbort)))
+        break;
+      const uint8_t* st = sX + s * kXStage;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        const int r = lane + 32 * j;
+        float part[4];
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+#pragma unroll
+          for (int hq = 0; hq < 2; ++hq) {
+            float acc = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t chunk = (uint32_t)(4 * hq + q);
+              const uint4 v = *reinterpret_cast<const uint4*>(
+                  st + hb * (kXStage / 2) + (r >> 3) * 1024 + (r & 7) * 128 +
+                  (((chunk ^ (uint32_t)(r & 7)) & 7u) << 4));
+              const __half2* h2 = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 f = __half22float2(h2[u]);
+                acc = fmaf(f.x, f.x, acc);
+                acc = fmaf(f.y, f.y, acc);
+              }
+            }
+            part[2 * hb + hq] = acc;
+          }
+        }
+        const float nu = sqrtf((part[0] + part[1]) + (part[2] + part[3]));
+        sNu[s * kRowsG + r] = nu;
+        const int64_t vrow = tile * kRowsG + r;
+        if (vrow < p.n) p.norms[vrow] = f32_to_f16_bits(nu);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&nu_full[s]);
+        ptx::mbar_arrive(&x_empty[s]);
+        // refill stage s with tile i + kStagesG once the MMA and every search warp are done
+        // with it
+        if (i + kStagesG < n_local) {
+          if (wait_g(&x_empty[s], (uint32_t)(i / kStagesG) & 1u, sAbort)) {
+            const int64_t nt = (int64_t)blockIdx.x + (int64_t)(i + kStagesG) * gridDim.x;
+            ptx::mbar_arrive_expect_tx(&x_full[s], kXStage);
+            ptx::tma_load_2d(sX + s * kXStage, &xmap, &x_full[s], 0, (int)(nt * kRowsG));
+            ptx::tma_load_2d(sX + s * kXStage + kXStage / 2, &xmap, &x_full[s], 64,
+                             (int)(nt * kRowsG));
+            issued = i + kStagesG + 1;
+          }
+        }
+      }
+      issued = __shfl_sync(0xffffffffu, issued, 0);
     }
+    if (lane == 0)  // copies in flight land before the CTA exits (bounded)
+      for (int t = issued - kStagesG < 0 ? 0 : issued - kStagesG; t < issued; ++t)
+        ptx::mbar_wait(&x_full[t % kStagesG], (uint32_t)(t / kStagesG) & 1u);
   } else if (warp == 1) {
     // ---- MMA issuer: D_b = X [Pi_hi ; 2^12 Pi_lo]^T ----
     if (lane == 0) {
@@ -282,45 +340,10 @@ __global__ void __launch_bounds__(kThreadsG, 1)
       const int64_t tile = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
       const int64_t vrow = tile * kRowsG + r;
       float nu = 0.f;
-      if (wg == 0) {  // the norm of row r from the swizzled x tile, handed to the others
-        fail = !wait_g(&x_full[s], ps, sAbort);
-        if (!fail) {
-          const uint8_t* st = sX + s * kXStage;
-          float part[4];
-#pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {
-#pragma unroll
-            for (int hq = 0; hq < 2; ++hq) {
-              float a = 0.f;
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const uint32_t chunk = (uint32_t)(4 * hq + q);
-                const uint4 v = *reinterpret_cast<const uint4*>(
-                    st + hb * (kXStage / 2) + (r >> 3) * 1024 + (r & 7) * 128 +
-                    (((chunk ^ (uint32_t)(r & 7)) & 7u) << 4));
-                const __half2* h2 = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const float2 f = __half22float2(h2[u]);
-                  a = fmaf(f.x, f.x, a);
-                  a = fmaf(f.y, f.y, a);
-                }
-              }
-              part[2 * hb + hq] = a;
-            }
-          }
-          nu = sqrtf((part[0] + part[1]) + (part[2] + part[3]));
-          sNu[s * kRowsG + r] = nu;
-          if (vrow < p.n) p.norms[vrow] = f32_to_f16_bits(nu);
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&nu_full[s]);
-      } else {
-        fail = !wait_g(&nu_full[s], ps, sAbort);
-        if (!fail) nu = sNu[s * kRowsG + r];
-      }
+      fail = !wait_g(&nu_full[s], ps, sAbort);
+      if (!fail) nu = sNu[s * kRowsG + r];
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&x_empty[s]);  // this warp no longer reads the stage
+      if (lane == 0) ptx::mbar_arrive(&x_empty[s]);  // this warp has read the stage's norms
       if (fail) break;
       const float rinv = nu > 0.f ? __frcp_rn(nu) : 0.f;
       // blocks 8 wg .. 8 wg + 7 in two halves of four: z = (D_hi + 2^-12 D_lo) / nu from the
@@ -395,7 +418,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
             // the exact winner
             if (!(d2 - d1 > 1.25e-4f * sqrtf(d2) + 6e-7f * d2 + 1e-8f))
               bi = rerank_exact(z[4 * bk], z[4 * bk + 1], z[4 * bk + 2], z[4 * bk + 3], ent[bk],
-                                h.slots, reinterpret_cast<const float4*>(p.cb));
+                                h.slots, sF32);
             const uint32_t ix = (uint32_t)bi & (kNG - 1);
             const uint32_t bit = (uint32_t)((4 * hb + bk) * kBG);
             rec[bit >> 5] |= ix << (bit & 31);
@@ -405,7 +428,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
 #pragma unroll
           for (int bk = 0; bk < 4; ++bk) {  // no usable index: exact brute force (fp32, L1/L2)
             const int bi = brute_exact(z[4 * bk], z[4 * bk + 1], z[4 * bk + 2], z[4 * bk + 3],
-                                       reinterpret_cast<const float4*>(p.cb));
+                                       sF32);
             const uint32_t ix = (uint32_t)bi & (kNG - 1);
             const uint32_t bit = (uint32_t)((4 * hb + bk) * kBG);
             rec[bit >> 5] |= ix << (bit & 31);
