@@ -77,10 +77,13 @@ struct GParams {
   uint16_t* norms;
 };
 
+// Bounded wait that gives up early when another role raised the abort flag.  try_wait suspends
+// the waiting warp in hardware between polls, so waiting warps take no issue slots from the
+// working ones.
 __device__ __forceinline__ bool wait_g(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  for (uint32_t it = 0; it < (ptx::kSpinLimit << 2); ++it) {
-    if (ptx::mbar_test(bar, parity)) return true;
-    if ((it & 63u) == 63u && *abort) return false;
+  for (uint32_t it = 0; it < ptx::kSpinLimit; ++it) {
+    if (ptx::mbar_try(bar, parity)) return true;
+    if ((it & 15u) == 15u && *abort) return false;
   }
   *abort = 1;
   return false;
