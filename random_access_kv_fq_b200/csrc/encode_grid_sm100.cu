@@ -94,8 +94,9 @@ __device__ __forceinline__ bool better_g(float v, int i, float bv, int bi) {
 }
 
 // Exact fp32 re-scoring of a block's candidate list (the rare case where the fixed-point
-// distances cannot separate the best two); lowest index on equal distances.
-__device__ __forceinline__ int rerank_exact(float z0, float z1, float z2, float z3, uint4 ent,
+// distances cannot separate the best two); lowest index on equal distances.  Out of line, so
+// that the common case branches around it instead of executing it under a predicate.
+__device__ __noinline__ int rerank_exact(float z0, float z1, float z2, float z3, uint4 ent,
                                             int slots, const float4* tbl) {
   const uint32_t words[4] = {ent.x, ent.y, ent.z, ent.w};
   float best = INFINITY;
