@@ -12,17 +12,13 @@
 //   warp 1       the rotation of each tile on the tensor cores, A = the x tile in shared memory,
 //                B = [Pi_hi ; 2^12 Pi_lo] (fp16 head and scaled residual of Pi), into one of two
 //                256-column accumulators in tensor memory
-//   warps 2-17   four warpgroups, thread (warpgroup w, row r): warpgroup 0 takes the norm of
-//                row r from the x tile and hands it over through shared memory; then every
-//                thread searches blocks 8w .. 8w + 7 of row r: z from the accumulator, the 8
-//                cells, the 8 index entries loaded at once from L2, and the candidates' squared
-//                distances from a shared table of 16-bit fixed-point codewords (8 bytes each:
-//                random 8-byte lookups run at almost twice the rate of 16-byte ones).  The
-//                fixed-point distance is within 2^-14 sqrt(d) of the exact one; a block whose
-//                best two approximate distances are closer than that bound is re-scored exactly
-//                in fp32 from the codebook in global memory (rare), so the result is the one of
-//                the exact fp32 search.  The warpgroups synchronise only through mbarriers.
-// The loads of tile i + 1 and i + 2 and their rotations overlap the search of tile i.
+//   warps 2-17   four warpgroups, thread (warpgroup w, row r): the norm of row r from the x
+//                tile (32 columns each, partial sums combined in a fixed order), then blocks
+//                8w .. 8w + 7 of row r: z from the accumulator, the 8 cells, the 8 index
+//                entries loaded at once from L2, the candidates from a shared fp32 codebook
+//                table; the 96 record bits are staged in shared memory and the tile's records
+//                leave with coalesced 16-byte stores.
+// The loads of tile i + 1 and its rotation overlap the search of tile i.
 #include <cstdint>
 
 #include <cuda.h>
@@ -49,24 +45,16 @@ constexpr int kXStage = kRowsG * kDG * 2;  // 32 KB: two [128 x 64] fp16 boxes
 
 __device__ unsigned int g_encg_wait_timeouts = 0;  // CTAs whose bounded waits gave up
 
-constexpr int kStagesG = 2;               // x tiles in flight
-
 struct GCfg {
   static constexpr int OFF_PI = 0;                      // [2 K halves][256 rows x 128 B]
-  static constexpr int OFF_X = OFF_PI + 2 * 256 * 128;  // [stages][2 boxes][128 x 128 B]
-  static constexpr int OFF_TBL = OFF_X + kStagesG * kXStage;  // N x 4 int16 codebook
-  static constexpr int OFF_F32 = OFF_TBL + kNG * 8;     // N x float4 codebook (exact scores)
-  static constexpr int OFF_NU = OFF_F32 + kNG * 16;     // [stages][128] norms
-  static constexpr int OFF_BAR = OFF_NU + kStagesG * kRowsG * 4;
+  static constexpr int OFF_X = OFF_PI + 2 * 256 * 128;  // [2 stages][2 boxes][128 x 128 B]
+  static constexpr int OFF_TBL = OFF_X + 2 * kXStage;   // N x float4 codebook
+  static constexpr int OFF_REC = OFF_TBL + kNG * 16;    // [128 rows][48 B] records
+  static constexpr int OFF_PART = OFF_REC + kRowsG * kPG;  // [4 quarters][128 rows] norm partials
+  static constexpr int OFF_BAR = OFF_PART + kRowsG * 4 * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
-
-// 16-bit fixed-point codeword coordinate: q = round(c 2^15) stored as u = q + 32768.  The float
-// 2 + u 2^-15 has the bit pattern 0x40000000 | (u << 7) (exponent of 2, 23-bit mantissa), so
-// c_q = q 2^-15 = float(bits) - 3 exactly, and z - c_q = (z + 3) - float(bits).
-__device__ __forceinline__ float fx_lo(uint32_t w) { return __uint_as_float(0x40000000u | ((w & 0xFFFFu) << 7)); }
-__device__ __forceinline__ float fx_hi(uint32_t w) { return __uint_as_float(0x40000000u | ((w >> 16) << 7)); }
 
 struct GParams {
   int64_t n;
@@ -89,36 +77,26 @@ __device__ __forceinline__ bool wait_g(uint64_t* bar, uint32_t parity, volatile 
   return false;
 }
 
+// Barrier among the 512 search threads that also ORs a predicate across them.
+__device__ __forceinline__ bool search_sync_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(kSearchThreads)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ bool better_g(float v, int i, float bv, int bi) {
   return v < bv || (v == bv && i < bi);
 }
 
-// Exact fp32 re-scoring of a block's candidate list (the rare case where the fixed-point
-// distances cannot separate the best two); lowest index on equal distances.  Out of line, so
-// that the common case branches around it instead of executing it under a predicate.
-__device__ __noinline__ int rerank_exact(float z0, float z1, float z2, float z3, uint4 ent,
-                                            int slots, const float4* tbl) {
-  const uint32_t words[4] = {ent.x, ent.y, ent.z, ent.w};
-  float best = INFINITY;
-  int bi = 0x7fffffff;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    if (q < slots) {
-      const int c = (int)((words[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
-      const float4 cv = tbl[c];
-      const float e0 = z0 - cv.x, e1 = z1 - cv.y, e2 = z2 - cv.z, e3 = z3 - cv.w;
-      const float dd = fmaf(e0, e0, fmaf(e1, e1, fmaf(e2, e2, e3 * e3)));
-      if (better_g(dd, c, best, bi)) {
-        best = dd;
-        bi = c;
-      }
-    }
-  }
-  return bi;
-}
-
 // Exact brute force over all N codewords (an index that does not describe this codebook).
-// Out of line: it only runs for such an index.
+// Out of line: it only runs for such an index, and the hot loop stays small.
 __device__ __noinline__ int brute_exact(float z0, float z1, float z2, float z3,
                                         const float4* tbl) {
   float best = INFINITY;
@@ -135,8 +113,6 @@ __device__ __noinline__ int brute_exact(float z0, float z1, float z2, float z3,
   return bi;
 }
 
-// 18 warps: with the register file split over four sub-partitions (five warps on two of them),
-// at most 96 registers per thread fit one CTA per SM.
 __global__ void __launch_bounds__(kThreadsG, 1)
     encode_grid_kernel(const __grid_constant__ CUtensorMap xmap, GParams p) {
   using C = GCfg;
@@ -145,14 +121,13 @@ __global__ void __launch_bounds__(kThreadsG, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sPi = smem + C::OFF_PI;
   uint8_t* sX = smem + C::OFF_X;
-  uint2* sTbl = reinterpret_cast<uint2*>(smem + C::OFF_TBL);
-  float4* sF32 = reinterpret_cast<float4*>(smem + C::OFF_F32);
-  float* sNu = reinterpret_cast<float*>(smem + C::OFF_NU);
-  uint64_t* x_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [3] x tile landed
-  uint64_t* x_empty = x_full + kStagesG;  // [3] rotation done and the stage's norms read
-  uint64_t* nu_full = x_empty + kStagesG; // [3] the stage's norms written (warpgroup 0)
-  uint64_t* z_full = nu_full + kStagesG;  // [2] rotation accumulator ready
-  uint64_t* z_empty = z_full + 2;         // [2] accumulator read (16 search warps)
+  float4* sTbl = reinterpret_cast<float4*>(smem + C::OFF_TBL);
+  uint8_t* sRec = smem + C::OFF_REC;
+  float* sPart = reinterpret_cast<float*>(smem + C::OFF_PART);
+  uint64_t* x_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [2] x tile landed
+  uint64_t* x_empty = x_full + 2;    // [2] rotation done and norms read (2 arrivals)
+  uint64_t* z_full = x_empty + 2;    // [2] rotation accumulator ready
+  uint64_t* z_empty = z_full + 2;    // [2] accumulator read (16 search warps)
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(z_empty + 2);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
 
@@ -167,12 +142,9 @@ __global__ void __launch_bounds__(kThreadsG, 1)
     ptx::tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < kStagesG; ++s) {
-      ptx::mbar_init(&x_full[s], 1);
-      ptx::mbar_init(&x_empty[s], 2 + kSearchThreads / 32);
-      ptx::mbar_init(&nu_full[s], 1);
-    }
     for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&x_full[s], 1);
+      ptx::mbar_init(&x_empty[s], 2);
       ptx::mbar_init(&z_full[s], 1);
       ptx::mbar_init(&z_empty[s], kSearchThreads / 32);
     }
@@ -219,14 +191,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int c = c0 + q * kThreadsG + tid;
-      if (c < kNG) {
-        auto fx = [](float x) -> uint32_t {
-          const float t = fminf(fmaxf(rintf(x * 32768.0f), -32768.0f), 32767.0f);
-          return (uint32_t)((int)t + 32768);
-        };
-        sTbl[c] = make_uint2(fx(v[q].x) | (fx(v[q].y) << 16), fx(v[q].z) | (fx(v[q].w) << 16));
-        sF32[c] = v[q];
-      }
+      if (c < kNG) sTbl[c] = v[q];
     }
   }
   ptx::fence_proxy_async_smem();
@@ -236,76 +201,22 @@ __global__ void __launch_bounds__(kThreadsG, 1)
   const uint32_t tmem = *sTmem;
 
   if (warp == 0) {
-    // ---- producer warp: x tiles into the ring (lane 0), and the norms of each landed tile
-    //      (four rows per lane, from the swizzled stage) handed to the search warps ----
-    if (lane == 0)
-      for (int i = 0; i < n_local && i < kStagesG; ++i) {
+    // ---- producer: x tiles into the two-stage ring ----
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n_local; ++i) {
+        const int s = i & 1;
+        if (i >= 2 && !wait_g(&x_empty[s], (uint32_t)((i >> 1) - 1) & 1u, sAbort)) break;
         const int64_t tile = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
-        ptx::mbar_arrive_expect_tx(&x_full[i], kXStage);
-        ptx::tma_load_2d(sX + i * kXStage, &xmap, &x_full[i], 0, (int)(tile * kRowsG));
-        ptx::tma_load_2d(sX + i * kXStage + kXStage / 2, &xmap, &x_full[i], 64,
+        ptx::mbar_arrive_expect_tx(&x_full[s], kXStage);
+        ptx::tma_load_2d(sX + s * kXStage, &xmap, &x_full[s], 0, (int)(tile * kRowsG));
+        ptx::tma_load_2d(sX + s * kXStage + kXStage / 2, &xmap, &x_full[s], 64,
                          (int)(tile * kRowsG));
+        issued = i + 1;
       }
-    int issued = n_local < kStagesG ? n_local : kStagesG;
-    for (int i = 0; i < n_local; ++i) {
-      const int s = i % kStagesG;
-      const int64_t tile = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
-      if (__any_sync(0xffffffffu, !wait_g(&x_full[s], (uint32_t)(i / kStagesG) & 1u, sAbort)))
-        break;
-      const uint8_t* st = sX + s * kXStage;
-#pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
-        const int r = lane + 32 * j;
-        float part[4];
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-#pragma unroll
-          for (int hq = 0; hq < 2; ++hq) {
-            float acc = 0.f;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t chunk = (uint32_t)(4 * hq + q);
-              const uint4 v = *reinterpret_cast<const uint4*>(
-                  st + hb * (kXStage / 2) + (r >> 3) * 1024 + (r & 7) * 128 +
-                  (((chunk ^ (uint32_t)(r & 7)) & 7u) << 4));
-              const __half2* h2 = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const float2 f = __half22float2(h2[u]);
-                acc = fmaf(f.x, f.x, acc);
-                acc = fmaf(f.y, f.y, acc);
-              }
-            }
-            part[2 * hb + hq] = acc;
-          }
-        }
-        const float nu = sqrtf((part[0] + part[1]) + (part[2] + part[3]));
-        sNu[s * kRowsG + r] = nu;
-        const int64_t vrow = tile * kRowsG + r;
-        if (vrow < p.n) p.norms[vrow] = f32_to_f16_bits(nu);
-      }
-      __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive(&nu_full[s]);
-        ptx::mbar_arrive(&x_empty[s]);
-        // refill stage s with tile i + kStagesG once the MMA and every search warp are done
-        // with it
-        if (i + kStagesG < n_local) {
-          if (wait_g(&x_empty[s], (uint32_t)(i / kStagesG) & 1u, sAbort)) {
-            const int64_t nt = (int64_t)blockIdx.x + (int64_t)(i + kStagesG) * gridDim.x;
-            ptx::mbar_arrive_expect_tx(&x_full[s], kXStage);
-            ptx::tma_load_2d(sX + s * kXStage, &xmap, &x_full[s], 0, (int)(nt * kRowsG));
-            ptx::tma_load_2d(sX + s * kXStage + kXStage / 2, &xmap, &x_full[s], 64,
-                             (int)(nt * kRowsG));
-            issued = i + kStagesG + 1;
-          }
-        }
-      }
-      issued = __shfl_sync(0xffffffffu, issued, 0);
+      for (int t = issued - 2 < 0 ? 0 : issued - 2; t < issued; ++t)  // in flight: land first
+        ptx::mbar_wait(&x_full[t & 1], (uint32_t)(t >> 1) & 1u);
     }
-    if (lane == 0)  // copies in flight land before the CTA exits (bounded)
-      for (int t = issued - kStagesG < 0 ? 0 : issued - kStagesG; t < issued; ++t)
-        ptx::mbar_wait(&x_full[t % kStagesG], (uint32_t)(t / kStagesG) & 1u);
   } else if (warp == 1) {
     // ---- MMA issuer: D_b = X [Pi_hi ; 2^12 Pi_lo]^T ----
     if (lane == 0) {
@@ -313,19 +224,19 @@ __global__ void __launch_bounds__(kThreadsG, 1)
       const uint32_t pi = ptx::smem_u32(sPi), xs = ptx::smem_u32(sX);
       int issued = 0;
       for (int i = 0; i < n_local; ++i) {
-        const int s = i % kStagesG, b = i & 1;
-        if (!wait_g(&x_full[s], (uint32_t)(i / kStagesG) & 1u, sAbort)) break;
-        if (i >= 2 && !wait_g(&z_empty[b], (uint32_t)((i >> 1) - 1) & 1u, sAbort)) break;
+        const int s = i & 1;
+        if (!wait_g(&x_full[s], (uint32_t)(i >> 1) & 1u, sAbort)) break;
+        if (i >= 2 && !wait_g(&z_empty[s], (uint32_t)((i >> 1) - 1) & 1u, sAbort)) break;
         ptx::tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          ptx::umma_f16(tmem + (uint32_t)(b * 256),
+          ptx::umma_f16(tmem + (uint32_t)(s * 256),
                         ptx::sdesc_kmajor_sw128(xs + s * kXStage + (ks >> 2) * (kXStage / 2) +
                                                 (ks & 3) * 32),
                         ptx::sdesc_kmajor_sw128(pi + (ks >> 2) * (256 * 128) + (ks & 3) * 32),
                         idesc, ks > 0 ? 1u : 0u);
         ptx::umma_commit(&x_empty[s]);
-        ptx::umma_commit(&z_full[b]);
+        ptx::umma_commit(&z_full[s]);
         issued = i + 1;
       }
       if (issued > 0) ptx::mbar_wait(&z_full[(issued - 1) & 1], (uint32_t)((issued - 1) >> 1) & 1u);
@@ -337,116 +248,127 @@ __global__ void __launch_bounds__(kThreadsG, 1)
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-    bool fail = false;
-    for (int i = 0; i < n_local && !fail; ++i) {
-      const int s = i % kStagesG, b = i & 1;
-      const uint32_t ps = (uint32_t)(i / kStagesG) & 1u;
+    const int st = tid - 64;                       // 0..511
+    for (int i = 0; i < n_local; ++i) {
+      const int s = i & 1;
       const int64_t tile = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
       const int64_t vrow = tile * kRowsG + r;
-      float nu = 0.f;
-      fail = !wait_g(&nu_full[s], ps, sAbort);
-      if (!fail) nu = sNu[s * kRowsG + r];
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&x_empty[s]);  // this warp has read the stage's norms
-      if (fail) break;
-      const float rinv = nu > 0.f ? __frcp_rn(nu) : 0.f;
-      // blocks 8 wg .. 8 wg + 7 in two halves of four: z = (D_hi + 2^-12 D_lo) / nu from the
-      // accumulator, the four cells, their index entries (loaded together), the candidates
-      fail = __any_sync(0xffffffffu, !wait_g(&z_full[b], (uint32_t)(i >> 1) & 1u, sAbort));
-      if (!fail) ptx::tc_fence_after();
-      const uint32_t dz = tmem + lane_base + (uint32_t)(b * 256 + 32 * wg);
-      uint32_t rec[3] = {0u, 0u, 0u};
+      // norm: squares of x[r][32 wg .. 32 wg + 31] from the swizzled tile
+      bool fail = !wait_g(&x_full[s], (uint32_t)(i >> 1) & 1u, sAbort);
+      if (!fail) {
+        const uint8_t* box = sX + s * kXStage + (wg >> 1) * (kXStage / 2);
+        float part = 0.f;
 #pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        float z[16];
-        if (!fail) {
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t chunk = (uint32_t)((wg & 1) * 4 + q);
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              box + (r >> 3) * 1024 + (r & 7) * 128 + (((chunk ^ (uint32_t)(r & 7)) & 7u) << 4));
+          const __half2* h2 = reinterpret_cast<const __half2*>(&v);
+          float a = 0.f;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 f = __half22float2(h2[u]);
+            a = fmaf(f.x, f.x, a);
+            a = fmaf(f.y, f.y, a);
+          }
+          part += a;
+        }
+        sPart[wg * kRowsG + r] = part;
+      }
+      if (search_sync_or(fail)) break;  // partials in place; the x stage is no longer read
+      if (st == 0) ptx::mbar_arrive(&x_empty[s]);
+      const float nu = sqrtf((sPart[r] + sPart[kRowsG + r]) + (sPart[2 * kRowsG + r] + sPart[3 * kRowsG + r]));
+      const float rinv = nu > 0.f ? __frcp_rn(nu) : 0.f;
+      if (wg == 0 && vrow < p.n) p.norms[vrow] = f32_to_f16_bits(nu);
+      // z of this thread's 8 blocks: (D_hi + 2^-12 D_lo) / nu
+      fail = !wait_g(&z_full[s], (uint32_t)(i >> 1) & 1u, sAbort);
+      float z[32];
+      if (!fail) {
+        ptx::tc_fence_after();
+        const uint32_t dz = tmem + lane_base + (uint32_t)(s * 256 + 32 * wg);
+#pragma unroll
+        for (int h16 = 0; h16 < 2; ++h16) {
           uint32_t hv[16], lv[16];
-          ptx::tmem_ld16(dz + 16 * hb, hv);
-          ptx::tmem_ld16(dz + 128 + 16 * hb, lv);
+          ptx::tmem_ld16(dz + 16 * h16, hv);
+          ptx::tmem_ld16(dz + 128 + 16 * h16, lv);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            z[e] = fmaf(__uint_as_float(lv[e]), kLoScaleG * rinv, __uint_as_float(hv[e]) * rinv);
+            z[16 * h16 + e] = fmaf(__uint_as_float(lv[e]), kLoScaleG * rinv,
+                                   __uint_as_float(hv[e]) * rinv);
         }
-        if (hb == 1) {  // the accumulator is read: the MMA of tile i + 2 may overwrite it
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&z_empty[b]);
-        }
-        if (fail || !(nu > 0.f)) continue;  // a zero vector keeps index 0 in every block
+        ptx::tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&z_empty[s]);
+      uint32_t rec[3] = {0u, 0u, 0u};
+      if (!fail && nu > 0.f) {  // a zero vector keeps index 0 in every block
         if (use_index) {
-          uint4 ent[4];
+          uint4 ent[8];
 #pragma unroll
-          for (int bk = 0; bk < 4; ++bk) {
+          for (int b = 0; b < 8; ++b) {
             int flat = 0, mul = 1;
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
-              const float t = (z[4 * bk + a] - h.lo) * h.inv_h;
+              const float t = (z[4 * b + a] - h.lo) * h.inv_h;
               int c = (int)floorf(t);
               c = c < 0 ? 0 : (c >= h.L ? h.L - 1 : c);
               flat += c * mul;
               mul *= h.L;
             }
             const uint8_t* e = p.index + h.cells_offset + (size_t)flat * h.entry_bytes;
-            ent[bk] = h.entry_bytes == 16
-                          ? __ldg(reinterpret_cast<const uint4*>(e))
-                          : make_uint4(__ldg(reinterpret_cast<const uint32_t*>(e)),
-                                       h.entry_bytes > 4 ? __ldg(reinterpret_cast<const uint32_t*>(e) + 1) : 0u,
-                                       h.entry_bytes > 8 ? __ldg(reinterpret_cast<const uint32_t*>(e) + 2) : 0u, 0u);
+            ent[b] = h.entry_bytes == 16
+                         ? __ldg(reinterpret_cast<const uint4*>(e))
+                         : make_uint4(__ldg(reinterpret_cast<const uint32_t*>(e)),
+                                      h.entry_bytes > 4 ? __ldg(reinterpret_cast<const uint32_t*>(e) + 1) : 0u,
+                                      h.entry_bytes > 8 ? __ldg(reinterpret_cast<const uint32_t*>(e) + 2) : 0u, 0u);
           }
 #pragma unroll
-          for (int bk = 0; bk < 4; ++bk) {
-            const uint32_t words[4] = {ent[bk].x, ent[bk].y, ent[bk].z, ent[bk].w};
-            const float z0 = z[4 * bk] + 3.f, z1 = z[4 * bk + 1] + 3.f;
-            const float z2 = z[4 * bk + 2] + 3.f, z3 = z[4 * bk + 3] + 3.f;
-            float d1 = INFINITY, d2 = INFINITY;
-            int i1 = 0;
+          for (int b = 0; b < 8; ++b) {
+            const uint32_t words[4] = {ent[b].x, ent[b].y, ent[b].z, ent[b].w};
+            float best = INFINITY;
+            int bi = 0;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               if (q < h.slots) {
                 const int c = (int)((words[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
-                const uint2 cw = sTbl[c];
-                const float u0 = z0 - fx_lo(cw.x), u1 = z1 - fx_hi(cw.x);
-                const float u2 = z2 - fx_lo(cw.y), u3 = z3 - fx_hi(cw.y);
-                const float dd = fmaf(u0, u0, fmaf(u1, u1, fmaf(u2, u2, u3 * u3)));
-                const bool lt = dd < d1;
-                d2 = lt ? d1 : fminf(d2, dd);
-                i1 = lt ? c : i1;
-                d1 = lt ? dd : d1;
+                const float4 cv = sTbl[c];
+                const float d0 = z[4 * b] - cv.x, d1 = z[4 * b + 1] - cv.y;
+                const float d2 = z[4 * b + 2] - cv.z, d3 = z[4 * b + 3] - cv.w;
+                const float dd = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
+                if (q == 0 || better_g(dd, c, best, bi)) {
+                  best = dd;
+                  bi = c;
+                }
               }
             }
-            int bi = i1;
-            // each fixed-point distance is within (2^-14 + 2^-21) sqrt(d) + 2.4e-7 d + 1e-9 of
-            // the exact one (codeword rounding 2^-16 per coordinate, z + 3 rounding 2^-23, fp32
-            // sums): unless the best two are closer than twice that, the approximate winner is
-            // the exact winner
-            if (!(d2 - d1 > 1.25e-4f * sqrtf(d2) + 6e-7f * d2 + 1e-8f))
-              bi = rerank_exact(z[4 * bk], z[4 * bk + 1], z[4 * bk + 2], z[4 * bk + 3], ent[bk],
-                                h.slots, sF32);
             const uint32_t ix = (uint32_t)bi & (kNG - 1);
-            const uint32_t bit = (uint32_t)((4 * hb + bk) * kBG);
+            const uint32_t bit = (uint32_t)(b * kBG);
             rec[bit >> 5] |= ix << (bit & 31);
             if ((bit & 31) + kBG > 32) rec[(bit >> 5) + 1] |= ix >> (32 - (bit & 31));
           }
         } else {
 #pragma unroll
-          for (int bk = 0; bk < 4; ++bk) {  // no usable index: exact brute force (fp32, L1/L2)
-            const int bi = brute_exact(z[4 * bk], z[4 * bk + 1], z[4 * bk + 2], z[4 * bk + 3],
-                                       sF32);
+          for (int b = 0; b < 8; ++b) {  // no usable index: exact brute force over the table
+            const int bi = brute_exact(z[4 * b], z[4 * b + 1], z[4 * b + 2], z[4 * b + 3], sTbl);
             const uint32_t ix = (uint32_t)bi & (kNG - 1);
-            const uint32_t bit = (uint32_t)((4 * hb + bk) * kBG);
+            const uint32_t bit = (uint32_t)(b * kBG);
             rec[bit >> 5] |= ix << (bit & 31);
             if ((bit & 31) + kBG > 32) rec[(bit >> 5) + 1] |= ix >> (32 - (bit & 31));
           }
         }
       }
-      if (fail) break;
-      if (vrow < p.n) {  // this warpgroup's three record words
-        uint32_t* dst = reinterpret_cast<uint32_t*>(p.codes + vrow * kPG) + 3 * wg;
-        dst[0] = rec[0];
-        dst[1] = rec[1];
-        dst[2] = rec[2];
-      }
+      uint32_t* rr = reinterpret_cast<uint32_t*>(sRec + r * kPG) + 3 * wg;
+      rr[0] = rec[0];
+      rr[1] = rec[1];
+      rr[2] = rec[2];
+      if (search_sync_or(fail)) break;  // the tile's records are staged
+      // coalesced 16-byte stores of the tile's records (contiguous in global memory)
+      const int64_t rows_here = (p.n - tile * kRowsG) < kRowsG ? (p.n - tile * kRowsG) : kRowsG;
+      const int n16 = (int)(rows_here * kPG / 16);
+      if (st < n16)
+        reinterpret_cast<uint4*>(p.codes + tile * kRowsG * kPG)[st] =
+            reinterpret_cast<const uint4*>(sRec)[st];
     }
   }
 
@@ -477,7 +399,7 @@ PFN_cuTensorMapEncodeTiled_v12000 grid_tensor_map_fn() {
 bool encode_grid_supported(fq_dtype xt, const Shape& s, const void* x, const void* codes,
                            const float* cb, const void* index) {
   if (xt != FQ_F16 || s.d != kDG || s.k != 4 || s.B != kBG || index == nullptr) return false;
-  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(codes) & 3) ||
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(codes) & 15) ||
       (reinterpret_cast<uintptr_t>(cb) & 15) || (reinterpret_cast<uintptr_t>(index) & 15))
     return false;
   int dev = 0, major = 0;
