@@ -358,3 +358,20 @@ def test_rate_identity_and_compression_points():
     assert fo.rate_bits_per_coord(4, 8) == 0.75  # sub-one-bit point
     assert fo.payload_bytes(64, 3, 64) == 17 and fo.payload_bytes(128, 4, 4096) == 48
     assert fo.payload_bytes(64, 4, 8) == 6 and fo.payload_bytes(64, 2, 8) == 12
+
+
+def test_high_k_codebooks_respect_the_shannon_bound_and_improve_on_their_start():
+    """The half- and full-vector codebooks (k = 32, 64 at N = 2^15, d' = 64): on held-out draws
+    of the block source their unit-vector MSE stays above the Shannon bound 4^-b (b = 15/k) and
+    below the deterministic initial codebook's (Lloyd refinement only lowers it); the full-vector
+    source is the unit sphere (every draw has norm 1)."""
+    rng = np.random.default_rng(777)
+    for k in (32, 64):
+        C = tables.codebook(64, k, 32768).astype(np.float64)
+        s = fo.sample_source_blocks(4000, 64, k, rng)
+        mse = fo.block_mse(s, C) * (64 // k)
+        mse0 = fo.block_mse(s, fo.init_codebook(64, k, 32768)) * (64 // k)
+        assert 4.0 ** (-15 / k) <= mse < mse0
+    full = fo.sample_source_blocks(100, 64, 64, rng)
+    np.testing.assert_allclose(np.linalg.norm(full, axis=1), 1.0, atol=1e-12)
+    np.testing.assert_allclose(fo.init_radii(64, 64, 16), 1.0)
