@@ -98,6 +98,15 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def tensor_peak():
+    """Dense fp16/bf16 tensor TFLOP/s: the measured burst figure (a kernel timed alone), else the
+    fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 # The sources a timed kernel is built from (its .cu files, the headers they include and the host
 # code that picks them): a recorded DRAM traffic figure only applies while these are unchanged.
 _COMMON = ["fq_device.cuh", "sm100_ptx.cuh", "fq_internal.h", "fq_api.cu", "codec_sm100.h"]
@@ -476,11 +485,34 @@ def attn_state(torch, fq, device, copies, rank):
         torch.cuda.synchronize()
         cs = torch.nn.functional.cosine_similarity(out, exact, dim=-1)
         return float(cs.mean()), float(cs.min())
-    return launch, step_bytes, cosine
+
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    lengths = torch.randint(1, w.tokens + 1, (w.batch,), dtype=torch.int32, device=device,
+                            generator=g)
+    lengths_app = torch.empty_like(lengths)
+    k_new = torch.randn((w.batch, w.hkv, w.d), generator=g, device=device).half()
+    v_new = torch.randn((w.batch, w.hkv, w.d), generator=g, device=device).half()
+
+    def launch_lengths():
+        fq.fq_attn_decode_lengths(q, lengths, kcs[0], kns[0], w.k_rate.k, w.k_rate.N, rk, ck,
+                                  vcs[0], vns[0], w.v_rate.k, w.v_rate.N, rv, cv,
+                                  scale=1 / math.sqrt(w.d), out=out, workspace=ws)
+
+    def launch_append():
+        fq.fq_attn_decode_append(q, k_new, v_new, lengths_app, kcs[1], kns[1], w.k_rate.k,
+                                 w.k_rate.N, rk, ck, vcs[1], vns[1], w.v_rate.k, w.v_rate.N, rv,
+                                 cv, scale=1 / math.sqrt(w.d), out=out, workspace=ws)
+
+    def reset_append(start):
+        lengths_app.fill_(start)
+    extra = {"lengths": lengths, "launch_lengths": launch_lengths,
+             "launch_append": launch_append, "reset_append": reset_append}
+    return launch, step_bytes, cosine, extra
 
 
 def attn_bench(torch, fq, timer, device, rank, hbm):
-    launch, attn_bytes, cosine = attn_state(torch, fq, device, 4, rank)
+    launch, attn_bytes, cosine, extra = attn_state(torch, fq, device, 4, rank)
     for c in range(4):
         launch(c)
     torch.cuda.synchronize()
@@ -492,12 +524,155 @@ def attn_bench(torch, fq, timer, device, rank, hbm):
     del graphs
     cmean, cmin = cosine()
     gbs = attn_bytes / (us * 1e-6) / 1e9
+    # random access: per-sequence lengths (random in [1, T]) and the step that appends its token
+    w = wl.ATTN
+    per_tok = attn_bytes / (w.batch * w.hkv * w.tokens)
+    us_len = _time_ms(torch, extra["launch_lengths"]) * 1e3
+    len_bytes = float(extra["lengths"].sum().item()) * w.hkv * per_tok
+    extra["reset_append"](w.tokens // 2)
+    us_app = _time_ms(torch, extra["launch_append"], reps=50) * 1e3
+    app_tokens = w.tokens // 2 + 26   # lengths advance by one per call: mean over the calls
+    app_bytes = w.batch * w.hkv * app_tokens * per_tok
     return {"workload": wl.ATTN.name, "us_per_step": round(us, 2), "bytes_per_step": attn_bytes,
             "reps": reps,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4)},
             "launches_per_step": 2,
-            "cosine_vs_exact_fp16_attention": {"mean": round(cmean, 5), "min": round(cmin, 5)}}
+            "cosine_vs_exact_fp16_attention": {"mean": round(cmean, 5), "min": round(cmin, 5)},
+            "lengths": {"us_per_step": round(us_len, 2), "bytes_per_step": int(len_bytes),
+                        "hbm_frac": round(len_bytes / (us_len * 1e-6) / 1e9 / hbm, 4),
+                        "lengths": "uniform random in [1, T] per sequence"},
+            "append": {"us_per_step": round(us_app, 2), "bytes_per_step": int(app_bytes),
+                       "hbm_frac": round(app_bytes / (us_app * 1e-6) / 1e9 / hbm, 4),
+                       "launches_per_step": 4,
+                       "step": "encode K, V of the new token into slot lengths[b], attend over "
+                               "lengths[b] + 1 tokens, advance lengths (from T/2)"}}
+
+
+# ----------------------------------------------------------------------------- the other rows
+
+def _time_ms(torch, fn, reps=None, target_s=0.2):
+    """Mean device ms of fn() (eager C-ABI calls on the current stream, CUDA events)."""
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if reps is None:
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        reps = max(3, min(200, int(target_s * 1e3 / max(e0.elapsed_time(e1), 1e-3))))
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def rows_bench(torch, fq, device, hbm, tflops):
+    """Throughput lines of the rows beyond the main codec step, each on a synthetic input of the
+    pages' workload shapes: half- and full-vector codes (the 34x end of the frontier), scalar
+    TurboQuant (k = 1) as the same-box baseline codec, the variants (BlockQuant rescale with a
+    stored rho, TurboQuant_prod), and random access (gather-decode of a token list, attention
+    over per-sequence lengths, the decode step that appends its own token)."""
+    from random_access_kv_fq_b200 import tables
+    out = {}
+    shape = wl.GPT2.cache
+    n, d = shape.n, shape.d
+    x = torch.from_numpy(wl.cache(shape, workers=min(32, len(os.sched_getaffinity(0))))).to(device)
+    rot64 = {dp: torch.from_numpy(tables.rotation(dp, wl.ROT_SEED_K)).to(device) for dp in (64, 66)}
+
+    def line(ms, vecs, alg_bytes, **extra):
+        gbs = alg_bytes / (ms * 1e-3) / 1e9
+        o = {"avg_us": round(ms * 1e3, 2), "vectors": vecs,
+             "Gvec_s": round(vecs / (ms * 1e-3) / 1e9, 4), "GBps_alg": round(gbs, 1),
+             "hbm_frac": round(gbs / hbm, 4)}
+        o.update(extra)
+        return o
+
+    # half- and full-vector codes on the GPT-2-shaped cache: tensor-core GEMM search
+    hk = {}
+    for k in (32, 64):
+        N = 32768
+        cbn = tables.codebook(64, k, N)
+        cb = torch.from_numpy(cbn).to(device)
+        ix = torch.from_numpy(fq.fq_build_search_index(cbn, 64, k, N, fq.FQ_INDEX_TENSOR, 0, 0)).to(device)
+        P = fq.fq_payload_bytes(64, k, N)
+        codes = torch.empty((n, P), dtype=torch.uint8, device=device)
+        norms = torch.empty((n,), dtype=torch.int16, device=device)
+        y = torch.empty((n, d), dtype=torch.float16, device=device)
+        me = _time_ms(torch, lambda: fq.fq_encode(x, rot64[64], cb, k, N, codes=codes, norms=norms,
+                                                  search_index=ix), reps=3)
+        md = _time_ms(torch, lambda: fq.fq_decode(codes, norms, rot64[64], cb, 64, k, N, y=y))
+        m = 64 // k
+        issued = 2.0 * n * m * N * (3 * k + 16)
+        search = 2.0 * n * m * N * k
+        hk[f"k{k}N{N}"] = {
+            "encode": line(me, n, n * (2 * d + P + 2), bound="tensor",
+                           tflops_issued=round(issued / (me * 1e-3) / 1e12, 1),
+                           tensor_frac=round(issued / (me * 1e-3) / 1e12 / tflops, 4),
+                           tflops_search=round(search / (me * 1e-3) / 1e12, 1)),
+            "decode": line(md, n, n * (P + 2 + 2 * d)),
+            "compression": {"pages_16_over_b": round(16 / (15 / k), 2),
+                            "true_fp16_over_record": round(2 * d / (P + 2), 2)}}
+        del codes, norms, y, ix
+    out["high_k"] = {"workload": wl.GPT2.name, "codebook": "Lloyd tables N = 2^15", **hk}
+
+    # scalar TurboQuant (k = 1, b = 2) on the same cache: the baseline codec of Thm 2
+    c1 = torch.from_numpy(tables.codebook(64, 1, 4)).to(device)
+    P1 = fq.fq_payload_bytes(64, 1, 4)
+    codes = torch.empty((n, P1), dtype=torch.uint8, device=device)
+    norms = torch.empty((n,), dtype=torch.int16, device=device)
+    y = torch.empty((n, d), dtype=torch.float16, device=device)
+    me = _time_ms(torch, lambda: fq.fq_encode(x, rot64[64], c1, 1, 4, codes=codes, norms=norms))
+    md = _time_ms(torch, lambda: fq.fq_decode(codes, norms, rot64[64], c1, 64, 1, 4, y=y))
+    out["scalar_turboquant_k1N4"] = {"encode": line(me, n, n * (2 * d + P1 + 2)),
+                                     "decode": line(md, n, n * (P1 + 2 + 2 * d)),
+                                     "path": "generic kernels (one warp per vector)"}
+
+    # variants on the same cache: BlockQuant rescale (k = 3, N = 64) and TurboQuant_prod (b = 2)
+    cb3 = torch.from_numpy(tables.codebook(66, 3, 64)).to(device)
+    P3 = fq.fq_payload_bytes(64, 3, 64)
+    st = {}
+    me = _time_ms(torch, lambda: st.__setitem__("r", fq.fq_encode_rho(x, rot64[66], cb3, 3, 64)))
+    codes3, norms3, rho = st["r"]
+    md = _time_ms(torch, lambda: fq.fq_decode_rescaled(codes3, norms3, rho, rot64[66], cb3, 64, 3,
+                                                       64, fq.FQ_RESCALE_MSE,
+                                                       out_dtype=torch.float16))
+    var = {"rescale_k3N64": {"encode_rho": line(me, n, n * (2 * d + P3 + 4)),
+                             "decode_mse_rule": line(md, n, n * (P3 + 4 + 2 * d))}}
+    c12 = torch.from_numpy(tables.codebook(64, 1, 2).ravel().copy()).to(device)
+    S = torch.from_numpy(np.random.default_rng(1234).standard_normal((64, 64)).astype(np.float32)).to(device)
+    me = _time_ms(torch, lambda: st.__setitem__("p", fq.fq_encode_prod(x, rot64[64], c12, S)))
+    pc, ps, pn, pg = st["p"]
+    md = _time_ms(torch, lambda: fq.fq_decode_prod(pc, ps, pn, pg, rot64[64], c12, S, 64,
+                                                   out_dtype=torch.float16))
+    rec = pc.shape[1] + ps.shape[1] + 4
+    var["turboquant_prod_b2"] = {"encode": line(me, n, n * (2 * d + rec)),
+                                 "decode": line(md, n, n * (rec + 2 * d))}
+    out["variants"] = var
+    del codes, norms, y, codes3, norms3, rho, pc, ps, pn, pg, x, st
+    torch.cuda.empty_cache()
+
+    # random access: gather-decode of a random eighth of a 4 M-record plane (d = 128, k = 4,
+    # N = 4096; the decode's cost does not depend on the record values, so they are random)
+    nr = 1 << 22
+    cb128 = torch.from_numpy(tables.codebook(128, 4, 4096)).to(device)
+    rot128 = torch.from_numpy(tables.rotation(128, wl.ROT_SEED_K)).to(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(5)
+    rcodes = torch.randint(0, 256, (nr, 48), dtype=torch.uint8, device=device, generator=g)
+    rnorms = torch.full((nr,), 0x3C00, dtype=torch.int16, device=device)   # fp16 1.0
+    ids = torch.randint(0, nr, (nr // 8,), dtype=torch.int64, device=device, generator=g)
+    yg = torch.empty((nr // 8, 128), dtype=torch.float16, device=device)
+    mg = _time_ms(torch, lambda: fq.fq_decode_gather(rcodes, rnorms, ids, rot128, cb128, 128, 4,
+                                                     4096, y=yg))
+    ra = {"gather_decode_d128_k4N4096": line(mg, nr // 8, (nr // 8) * (48 + 2 + 8 + 256),
+                                             ids=nr // 8, plane=nr)}
+    del rcodes, rnorms, ids, yg
+    out["random_access"] = ra
+    return out
 
 
 # ----------------------------------------------------------------------------- arms
@@ -604,6 +779,9 @@ def run_gpu(args):
     # ---- fused attention step
     if not args.no_attn:
         result["attn"] = attn_bench(torch, fq, timer, device, rank, hbm)
+    # ---- the rows beyond the main step (high-k, scalar baseline, variants, random access)
+    if not args.no_configs and not args.tokens:
+        result["rows"] = rows_bench(torch, fq, device, hbm, tensor_peak()[0])
     bad = fq.fq_wait_status(clear=True)
     if bad:
         raise RuntimeError(f"{bad} CTAs gave up a bounded wait during the bench")

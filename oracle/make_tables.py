@@ -39,6 +39,8 @@ CODEBOOKS = [
     (64, 64, 32768, 1, 20, 4 * 32768),
 ]
 CODEBOOK_SEED = 101
+# scalar Lloyd-Max levels of the coordinate law (k = 1, TurboQuant notes sec. 3.1): (d, N1)
+SCALAR = [(64, 2), (64, 4), (64, 16)]
 
 
 def rot_name(dp, seed):
@@ -82,6 +84,15 @@ def main(argv=None):
                           "seconds": round(time.time() - t0, 1)}
         print(name, manifest[name], flush=True)
         json.dump(manifest, open(man_path, "w"), indent=1, sort_keys=True)
+    for d, N1 in SCALAR:
+        name = cb_name(d, 1, N1)
+        if args.only is not None and name not in args.only:
+            continue
+        c1 = np.sort(fo.scalar_lloyd(d, N1))
+        np.save(os.path.join(OUT, name + ".npy"), c1.astype(np.float32)[:, None])
+        manifest[name] = {"kind": "scalar codebook", "d": d, "N": N1,
+                          "mse_per_coord": fo.scalar_mse_per_coord(c1, d)}
+        print(name, manifest[name], flush=True)
     json.dump(manifest, open(man_path, "w"), indent=1, sort_keys=True)
 
 
