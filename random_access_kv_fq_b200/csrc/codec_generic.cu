@@ -441,7 +441,7 @@ cudaError_t launch_encode_generic(const void* x, fq_dtype xt, int64_t n, const S
                                   AppendMap map, uint16_t* rho) {
   // without an index and with a codebook small enough for a per-thread brute force: the tiled
   // kernel; otherwise one warp per vector (candidate lists, or lanes striding over codewords)
-  if (index == nullptr && s.N <= 1024) {
+  if (index == nullptr && s.N <= 1024 && n >= 2048) {
     const int rn = (s.dp + 15) / 16 <= 4 ? 4 : ((s.dp + 15) / 16 <= 8 ? 8 : 16);
     const size_t smem = encode_tiled_smem(s, rn);
     if (smem <= 200 * 1024) {
