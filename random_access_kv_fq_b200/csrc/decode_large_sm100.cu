@@ -209,18 +209,23 @@ __global__ void __launch_bounds__(kThreadsDL, 1)
     if (bulk_tile(i)) {  // from the double buffer (bounded wait for the copy)
       const bool ok = ptx::mbar_wait(&rec_full[pipe * 2 + (i & 1)], (uint32_t)(i >> 1) & 1u);
       if (!ok) *sAbort = 1;
-      const uint4* src = reinterpret_cast<const uint4*>(sRec + (i & 1) * C::REC + lt * C::P);
+      // a record is P = 4 B bytes: 16-byte reads when P is a multiple of 16 (B % 4 == 0),
+      // else 4-byte reads (every record starts on a 4-byte boundary)
+      const uint8_t* rp = sRec + (i & 1) * C::REC + lt * C::P;
+      if constexpr (B % 4 == 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(rp);
 #pragma unroll
-      for (int q = 0; q < B / 4; ++q) {
-        const uint4 v = src[q];
-        w[4 * q] = v.x;
-        w[4 * q + 1] = v.y;
-        w[4 * q + 2] = v.z;
-        w[4 * q + 3] = v.w;
+        for (int q = 0; q < B / 4; ++q) {
+          const uint4 v = src[q];
+          w[4 * q] = v.x;
+          w[4 * q + 1] = v.y;
+          w[4 * q + 2] = v.z;
+          w[4 * q + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < B; ++q) w[q] = reinterpret_cast<const uint32_t*>(rp)[q];
       }
-#pragma unroll
-      for (int q = (B / 4) * 4; q < B; ++q)
-        w[q] = reinterpret_cast<const uint32_t*>(sRec + (i & 1) * C::REC + lt * C::P)[q];
       w[B] = 0u;
       nu = f16_bits_to_f32(reinterpret_cast<const uint16_t*>(sNrm + (i & 1) * C::NRM)[lt]);
       return;
