@@ -219,17 +219,29 @@ __global__ void __launch_bounds__(kDecThreads)
       scale[tid] = r >= 0 ? f16_bits_to_f32(norms[r]) : (r == -2 ? __int_as_float(0x7fc00000) : 0.f);
     }
     __syncthreads();
-    // a6 + a7: unpack each index and gather its codeword into the concatenated zhat
+    // a6: unpack each index once (into the rows' first columns of ps, which is free here)
+    int* pid = reinterpret_cast<int*>(ps);
+    const bool fit = kTileR * s.m <= kKChunk * 16 * RN;
+    if (fit)
+      for (int e = tid; e < kTileR * s.m; e += kDecThreads) {
+        const int r = e / s.m, j = e - r * s.m;
+        const int64_t rec = src[r];
+        pid[e] = rec >= 0 ? record_index(codes + rec * s.P, j, s.B) : -1;
+      }
+    __syncthreads();
+    // a7: gather the codewords into the concatenated zhat (consecutive threads read consecutive
+    // coordinates of a codeword)
     for (int e = tid; e < kTileR * s.dp; e += kDecThreads) {
       const int r = e / s.dp, c = e - r * s.dp;
-      const int64_t rec = src[r];
-      float v = 0.f;
-      if (rec >= 0) {
-        const int j = c / s.k;
-        const int idx = record_index(codes + rec * s.P, j, s.B);
-        v = __ldg(cb + (size_t)idx * s.k + (c - j * s.k));
+      const int j = c / s.k;
+      int idx;
+      if (fit) {
+        idx = pid[r * s.m + j];
+      } else {
+        const int64_t rec = src[r];
+        idx = rec >= 0 ? record_index(codes + rec * s.P, j, s.B) : -1;
       }
-      zs[r * zstride + c] = v;
+      zs[r * zstride + c] = idx >= 0 ? __ldg(cb + (size_t)idx * s.k + (c - j * s.k)) : 0.f;
     }
     __syncthreads();
     if (rs.rho != nullptr && tid < kTileR && src[tid] >= 0) {
@@ -290,6 +302,31 @@ __global__ void __launch_bounds__(kDecThreads)
 // searches all N codewords (from shared memory when they fit), lowest index on ties, and the
 // records are packed byte by byte.
 constexpr int kEncCbSmem = 8192;  // codebook floats kept in shared memory
+
+// Nearest of N codewords of K coordinates to the block zb (direct-form squared distances, the
+// block in registers; strict < over increasing c keeps the lowest index on ties).
+template <int K>
+__device__ __forceinline__ int nearest_small(const float* zb, const float* cbp, int N) {
+  float z[K];
+#pragma unroll
+  for (int q = 0; q < K; ++q) z[q] = zb[q];
+  float best = INFINITY;
+  int bi = 0;
+#pragma unroll 4
+  for (int c = 0; c < N; ++c) {
+    float dist = 0.f;
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      const float t = z[q] - cbp[c * K + q];
+      dist = fmaf(t, t, dist);
+    }
+    if (dist < best) {
+      best = dist;
+      bi = c;
+    }
+  }
+  return bi;
+}
 
 template <typename TX, int RN>
 __global__ void __launch_bounds__(kDecThreads)
@@ -368,18 +405,27 @@ __global__ void __launch_bounds__(kDecThreads)
     for (int e = tid; e < kTileR * s.m; e += kDecThreads) {
       const int r = e / s.m, j = e - r * s.m;
       const float* zb = zs + r * zstride + j * s.k;
-      float best = INFINITY;
-      int bi = 0;
-      for (int c = 0; c < s.N; ++c) {
-        const float* cw = cbp + (size_t)c * s.k;
-        float dist = 0.f;
-        for (int q = 0; q < s.k; ++q) {
-          const float t = zb[q] - cw[q];
-          dist = fmaf(t, t, dist);
-        }
-        if (dist < best) {
-          best = dist;
-          bi = c;
+      int bi;
+      switch (s.k) {
+        case 1: bi = nearest_small<1>(zb, cbp, s.N); break;
+        case 2: bi = nearest_small<2>(zb, cbp, s.N); break;
+        case 3: bi = nearest_small<3>(zb, cbp, s.N); break;
+        case 4: bi = nearest_small<4>(zb, cbp, s.N); break;
+        default: {
+          float best = INFINITY;
+          bi = 0;
+          for (int c = 0; c < s.N; ++c) {
+            const float* cw = cbp + (size_t)c * s.k;
+            float dist = 0.f;
+            for (int q = 0; q < s.k; ++q) {
+              const float t = zb[q] - cw[q];
+              dist = fmaf(t, t, dist);
+            }
+            if (dist < best) {
+              best = dist;
+              bi = c;
+            }
+          }
         }
       }
       ids[r * s.m + j] = nus[r] > 0.f ? bi : 0;
