@@ -554,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
-  if constexpr (B <= 4) {  // N <= 16: brute force from registers (same result as any index)
+  if constexpr (B <= 4 && !GRID) {  // N <= 16 without an index: brute force from registers
     SearchRegs<K, B> sr;
     sr.load(tbl);
     run(sr);
@@ -630,7 +630,9 @@ cudaError_t launch_kernel(const void* x, const EncParams& p, cudaStream_t st) {
 
 template <int K, int DP, int B>
 cudaError_t launch_rate(const void* x, const EncParams& p, cudaStream_t st) {
-  if (p.index != nullptr && B > 4) return launch_kernel<K, DP, B, true>(x, p, st);
+  // with an index, codebooks of 16 codewords and more search their grid candidate lists (3
+  // candidates at N = 16 against 16 from registers); smaller ones keep the register brute force
+  if (p.index != nullptr && B >= 4) return launch_kernel<K, DP, B, true>(x, p, st);
   return launch_kernel<K, DP, B, false>(x, p, st);
 }
 
