@@ -111,10 +111,10 @@ def tensor_peak():
 # code that picks them): a recorded DRAM traffic figure only applies while these are unchanged.
 _COMMON = ["fq_device.cuh", "sm100_ptx.cuh", "fq_internal.h", "fq_api.cu", "codec_sm100.h"]
 KERNEL_SOURCES = {
-    ("encode", 64): ["encode_sm100.cu", "codec_generic.cu"],
-    ("decode", 64): ["decode_sm100.cu", "codec_generic.cu"],
-    ("encode", 128): ["encode_large_sm100.cu", "codec_generic.cu"],
-    ("decode", 128): ["decode_large_sm100.cu", "codec_generic.cu"],
+    ("encode", 64): ["encode_sm100.cu"],
+    ("decode", 64): ["decode_sm100.cu"],
+    ("encode", 128): ["encode_grid_sm100.cu", "encode_large_sm100.cu"],
+    ("decode", 128): ["decode_large_sm100.cu"],
     ("attn", 64): ["attn_sm100.cu", "attn.cu"],
 }
 
