@@ -216,6 +216,19 @@ def test_large_grid_index_for_another_codebook_falls_back_to_brute_force():
     par.check_norms(par.to_np(norms), enc)
 
 
+@pytest.mark.parametrize("L,c", [(8, 4), (12, 6), (16, 5)])
+def test_large_grid_index_of_other_shapes(L, c):
+    """d = 128, N = 4096 with top-c indexes other than 16 cells per axis x 8 candidates: the grid
+    kernel's general candidate loop, against the oracle's own top-c search."""
+    d = 128
+    rate = wl.Rate(4, 4096, "top", L, c)
+    rot, cb = tables.rotation(d, wl.ROT_SEED_K), tables.codebook(d, 4, 4096)
+    x = wl.rows_of(wl.LARGE.cache, np.arange(0, wl.LARGE.cache.n, wl.LARGE.cache.n // 1100)[:1100])
+    x = np.array(x)
+    x[5] = 0
+    run_codec(x, rot, cb, rate, d)
+
+
 @pytest.mark.parametrize("dp,k,N", [(64, 2, 16), (66, 3, 64), (64, 4, 8), (64, 2, 256)])
 def test_fast_and_generic_paths_meet_parity_on_the_same_rows(dp, k, N):
     """A 16-byte-aligned fp16 input takes the tensor-core kernel; the same rows behind a
