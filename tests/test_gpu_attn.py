@@ -100,9 +100,10 @@ def test_attention_empty_context_is_zero():
     assert torch.count_nonzero(out) == 0
 
 
-def test_attention_full_size_sampled():
-    """The full decode step (B16, Hq32/Hkv4, T32768) on a GPU-encoded cache; sampled (b, kv
-    head) groups checked against the oracle over the oracle-decoded GPU records."""
+def test_attention_full_size_all_groups():
+    """The full decode step (B16, Hq32/Hkv4, T32768) on a GPU-encoded cache; every (b, kv head)
+    group (so every context split of the launch) checked against the oracle over the
+    oracle-decoded GPU records."""
     w = wl.ATTN
     shape = wl.attn_cache_shape(w)
     dpk, dpv = fo.padded_dim(w.d, 2), fo.padded_dim(w.d, 3)
@@ -120,7 +121,7 @@ def test_attention_full_size_sampled():
     torch.cuda.synchronize()
     out = par.to_np(out)
     G = w.hq // w.hkv
-    for b, g in ((0, 0), (7, 3), (15, 1)):
+    for b, g in ((b, g) for b in range(w.batch) for g in range(w.hkv)):
         Kc = fo.CompressedKV(par.to_np(tensors["K"][0][b:b + 1, g:g + 1]),
                              par.to_np(tensors["K"][1][b:b + 1, g:g + 1]).view(np.float16),
                              rk, ck, 2, 16)
