@@ -540,7 +540,7 @@ class CompressedKV:
 
 def attention_decoded(q: np.ndarray, Kc: CompressedKV, Vc: CompressedKV, d: int,
                       scale: float) -> np.ndarray:
-    """Attention over the fully decoded caches (the reference the kernel is judged by)."""
+    """Attention over the fully decoded caches (what the CUDA attention is checked against)."""
     Bn, Hkv, T, _ = Kc.codes.shape
     Kh = decode(Kc.codes.reshape(-1, Kc.codes.shape[-1]), Kc.norms.reshape(-1), Kc.rot,
                 Kc.codebook, d, Kc.k, Kc.N).reshape(Bn, Hkv, T, d)
