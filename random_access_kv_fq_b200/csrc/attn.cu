@@ -243,9 +243,11 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AttnArgs a) {
 
 }  // namespace
 
-int attn_splits(int B, int Hkv, int64_t T) {
+int attn_splits(int B, int Hkv, int64_t T, bool ragged) {
   int64_t pairs = (int64_t)B * Hkv;
-  int64_t want = kTargetCtas / pairs;
+  // With per-sequence lengths the splits past a sequence's end exit at once and the step lasts
+  // as long as the busiest split: twice as many, half as long.
+  int64_t want = (ragged ? 2 * kTargetCtas : kTargetCtas) / pairs;
   int64_t tiles = (T + kSplitGrain - 1) / kSplitGrain;
   if (want > tiles) want = tiles;
   if (want < 1) want = 1;

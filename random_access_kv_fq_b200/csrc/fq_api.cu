@@ -161,7 +161,7 @@ fq_status attn_prepare(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int
   a->lengths_out = nullptr;
   a->splits = attn_splits(B, Hkv, T);
   a->tokens_per_split = attn_tokens_per_split(T, a->splits);
-  *need = attn_partials_bytes(B, Hq, a->splits, a->vs.dp);
+  *need = attn_partials_bytes(B, Hq, attn_splits(B, Hkv, T, true), a->vs.dp);
   if (attn_smem_bytes(*a) > 200 * 1024) return FQ_ERR_UNSUPPORTED;
   return FQ_OK;
 }
@@ -174,8 +174,7 @@ size_t fq_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int d, int kV)
   Shape ks, vs;
   if (attn_shapes(B, Hq, Hkv, T, d, 1, 2, kV, 2, &ks, &vs) != FQ_OK) return 0;
   if (T == 0) return 0;
-  int splits = attn_splits(B, Hkv, T);
-  return attn_partials_bytes(B, Hq, splits, vs.dp);
+  return attn_partials_bytes(B, Hq, attn_splits(B, Hkv, T, true), vs.dp);
 }
 
 fq_status fq_attn_decode(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int d,
@@ -242,6 +241,8 @@ fq_status fq_attn_decode_lengths(const uint16_t* q, int B, int Hq, int Hkv, int6
   if (!aligned(workspace, 16)) return FQ_ERR_ALIGNMENT;
   a.partials = static_cast<float*>(workspace);
   a.lengths = lengths;
+  a.splits = attn_splits(B, Hkv, T, true);
+  a.tokens_per_split = attn_tokens_per_split(T, a.splits);
   return from_cuda(launch_attn(a, cs));
 }
 
@@ -273,6 +274,8 @@ fq_status fq_attn_decode_append(const uint16_t* q, const uint16_t* k_new, const 
   if (e != cudaSuccess) return FQ_ERR_CUDA;
   a.partials = static_cast<float*>(workspace);
   a.lengths = lengths;
+  a.splits = attn_splits(B, Hkv, T, true);
+  a.tokens_per_split = attn_tokens_per_split(T, a.splits);
   a.length_bias = 1;
   a.lengths_out = lengths;
   return from_cuda(launch_attn(a, cs));

@@ -162,7 +162,10 @@ fq_status attn_prepare(const uint16_t* q, int B, int Hq, int Hkv, int64_t T, int
                        const float* rotK, const float* cbK, const uint8_t* v_codes,
                        const uint16_t* v_norms, int kV, int NV, const float* rotV,
                        const float* cbV, float scale, float* out, AttnArgs* a, size_t* need);
-int attn_splits(int B, int Hkv, int64_t T);
+// Context splits per (batch, kv head): about three 128-token-tile CTAs per SM, twice as many
+// when per-sequence lengths leave the splits past each sequence's end empty (ragged).  The
+// workspace is sized for the ragged count, which is never the smaller.
+int attn_splits(int B, int Hkv, int64_t T, bool ragged = false);
 int64_t attn_tokens_per_split(int64_t T, int splits);
 size_t attn_partials_bytes(int B, int Hq, int splits, int dpV);
 size_t attn_smem_bytes(const AttnArgs& a);
