@@ -629,19 +629,26 @@ def rows_bench(torch, fq, device, hbm, tflops):
     md = _time_ms(torch, lambda: fq.fq_decode(codes, norms, rot64[64], c1, 64, 1, 4, y=y))
     out["scalar_turboquant_k1N4"] = {"encode": line(me, n, n * (2 * d + P1 + 2)),
                                      "decode": line(md, n, n * (P1 + 2 + 2 * d)),
-                                     "path": "generic kernels (one warp per vector)"}
+                                     "path": "generic kernels (tiled FFMA rotation)"}
 
     # variants on the same cache: BlockQuant rescale (k = 3, N = 64) and TurboQuant_prod (b = 2)
-    cb3 = torch.from_numpy(tables.codebook(66, 3, 64)).to(device)
+    cb3n = tables.codebook(66, 3, 64)
+    cb3 = torch.from_numpy(cb3n).to(device)
+    ix3 = torch.from_numpy(fq.fq_build_search_index(cb3n, 64, 3, 64, fq.FQ_INDEX_EXACT, 20,
+                                                    8)).to(device)  # the GPT-2 k3N64 search
     P3 = fq.fq_payload_bytes(64, 3, 64)
     st = {}
-    me = _time_ms(torch, lambda: st.__setitem__("r", fq.fq_encode_rho(x, rot64[66], cb3, 3, 64)))
+    me = _time_ms(torch, lambda: st.__setitem__("r", fq.fq_encode_rho(x, rot64[66], cb3, 3, 64,
+                                                                       search_index=ix3)))
     codes3, norms3, rho = st["r"]
     md = _time_ms(torch, lambda: fq.fq_decode_rescaled(codes3, norms3, rho, rot64[66], cb3, 64, 3,
                                                        64, fq.FQ_RESCALE_MSE,
                                                        out_dtype=torch.float16))
     var = {"rescale_k3N64": {"encode_rho": line(me, n, n * (2 * d + P3 + 4)),
-                             "decode_mse_rule": line(md, n, n * (P3 + 4 + 2 * d))}}
+                             "decode_mse_rule": line(md, n, n * (P3 + 4 + 2 * d)),
+                             "path": "the d = 64 tensor-core kernels: encode with the exact grid "
+                                     "index (L20 c8) and rho, decode with S(rho) in the norm "
+                                     "scale"}}
     c12 = torch.from_numpy(tables.codebook(64, 1, 2).ravel().copy()).to(device)
     S = torch.from_numpy(np.random.default_rng(1234).standard_normal((64, 64)).astype(np.float32)).to(device)
     me = _time_ms(torch, lambda: st.__setitem__("p", fq.fq_encode_prod(x, rot64[64], c12, S)))

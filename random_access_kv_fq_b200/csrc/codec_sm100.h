@@ -10,9 +10,10 @@ namespace sm100 {
 // True when the fast kernel handles this call (shape, dtype and pointer alignment).
 bool encode_supported(fq_dtype xt, const Shape& s, const void* x, const void* codes,
                       const void* norms);
+// rho != nullptr: also <z, zhat> per vector in fp16 (the rescale variant's stored rho).
 cudaError_t launch_encode(const void* x, fq_dtype xt, int64_t n, const Shape& s,
                           const float* rot, const float* cb, uint8_t* codes, uint16_t* norms,
-                          const void* index, cudaStream_t st);
+                          const void* index, cudaStream_t st, uint16_t* rho = nullptr);
 
 // Large codebooks (d = 128, k = 4, N = 512 .. 4096, no index): tensor-core brute force.
 bool encode_large_supported(fq_dtype xt, const Shape& s, const void* x, const void* codes,
@@ -47,9 +48,11 @@ cudaError_t launch_decode_large(const uint8_t* codes, const uint16_t* norms, int
 
 bool decode_supported(fq_dtype yt, const Shape& s, const void* codes, const void* norms,
                       const void* y);
+// rho != nullptr: the rescale variant, y = S nu (Pi^T zbar) with S of `rule` (FQ_RESCALE_*).
 cudaError_t launch_decode(const uint8_t* codes, const uint16_t* norms, int64_t n,
                           const Shape& s, const float* rot, const float* cb, void* y,
-                          fq_dtype yt, cudaStream_t st);
+                          fq_dtype yt, cudaStream_t st, const uint16_t* rho = nullptr,
+                          int rule = 0);
 
 }  // namespace sm100
 }  // namespace fq

@@ -75,7 +75,8 @@ struct DecCfg {
   static constexpr int OFF_OUT = ((B_BYTES + 1023) / 1024) * 1024;
   static constexpr int OFF_RING = OFF_OUT + 4 * 2 * OUT_TILE;
   static constexpr int OFF_CB = OFF_RING + kStages * STAGE;
-  static constexpr int OFF_BAR = OFF_CB + N * REP * CBE;
+  static constexpr int OFF_CC = OFF_CB + N * REP * CBE;  // |c|^2 per codeword (the rescale)
+  static constexpr int OFF_BAR = OFF_CC + N * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -175,6 +176,8 @@ struct DecArgs {
   const uint8_t* codes;
   const uint16_t* norms;
   void* y;
+  const uint16_t* rho;  // the rescale variant: stored rho per record (fp16) and the S rule
+  int rule;
 };
 
 // Gather of one half of a zhat row into the tensor-memory A operand (this thread's lane): half 0
@@ -238,7 +241,7 @@ __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <int K, int DP, int B, bool F16>
+template <int K, int DP, int B, bool F16, bool RS>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_ws_kernel(const __grid_constant__ CUtensorMap ymap, DecArgs p) {
   using C = DecCfg<K, DP, B, F16>;
@@ -448,6 +451,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(b_ready);
+      if constexpr (RS) {  // |c|^2 per codeword for the MSE rule's |zbar|^2
+        float* sCc = reinterpret_cast<float*>(smem + C::OFF_CC);
+        for (int c = t; c < C::N; c += kEpiThreads) {
+          float cc = 0.f;
+#pragma unroll
+          for (int a = 0; a < K; ++a) {
+            const float v = __ldg(p.cb + (size_t)c * K + a);
+            cc = fmaf(v, v, cc);
+          }
+          sCc[c] = cc;
+        }
+        named_sync(2, kEpiThreads);
+      }
     }
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;
@@ -463,6 +479,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         nu = f16_bits_to_f32(direct(rows) ? p.norms[tile * kRows + r]
                                           : *reinterpret_cast<const uint16_t*>(
                                                 sRing + s * C::STAGE + C::REC + 2 * r));
+      if constexpr (RS) {
+        // Block Sphere VQ key design 3: y = S nu (Pi^T zbar), S from the stored rho and, for
+        // the MSE rule, |zbar|^2 = sum_j |c_j|^2 over the record's codewords
+        if (r < rows) {
+          uint32_t w[NW];
+          if (direct(rows)) read_rec_global<P>(p.codes + (tile * kRows + r) * P, w);
+          else read_rec<P>(sRing + s * C::STAGE, (uint32_t)(r * P), w);
+          const float* sCc = reinterpret_cast<const float*>(smem + C::OFF_CC);
+          float zz = 0.f;
+#pragma unroll
+          for (int j = 0; j < C::M; ++j) zz += sCc[field<B>(w, j)];
+          const float rho = f16_bits_to_f32(p.rho[tile * kRows + r]);
+          const float S = p.rule == FQ_RESCALE_MSE ? rho / zz
+                          : p.rule == FQ_RESCALE_UNBIASED ? 1.f / rho : 1.f;
+          nu *= S;
+        }
+      }
       ptx::mbar_arrive(&r_empty[s]);
       ok = wait_ab(&d_full[b], (uint32_t)(i >> 1) & 1u, sAbort);
       if (__any_sync(0xffffffffu, !ok)) break;
@@ -550,7 +583,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_fn() {
   return fn;
 }
 
-template <int K, int DP, int B, bool F16>
+template <int K, int DP, int B, bool F16, bool RS>
 cudaError_t launch_ws(const DecArgs& p, cudaStream_t st) {
   using C = DecCfg<K, DP, B, F16>;
   // output y [n x 64] (fp16 rows of 128 B, fp32 rows of 256 B), stored in boxes of 32 rows and
@@ -566,7 +599,7 @@ cudaError_t launch_ws(const DecArgs& p, cudaStream_t st) {
          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = decode_ws_kernel<K, DP, B, F16>;
+  auto kern = decode_ws_kernel<K, DP, B, F16, RS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -578,19 +611,25 @@ cudaError_t launch_ws(const DecArgs& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int K, int DP, bool F16>
-cudaError_t by_b(int B, const DecArgs& p, cudaStream_t st) {
+template <int K, int DP, bool F16, bool RS>
+cudaError_t by_b_rs(int B, const DecArgs& p, cudaStream_t st) {
   switch (B) {
-    case 1: return launch_ws<K, DP, 1, F16>(p, st);
-    case 2: return launch_ws<K, DP, 2, F16>(p, st);
-    case 3: return launch_ws<K, DP, 3, F16>(p, st);
-    case 4: return launch_ws<K, DP, 4, F16>(p, st);
-    case 5: return launch_ws<K, DP, 5, F16>(p, st);
-    case 6: return launch_ws<K, DP, 6, F16>(p, st);
-    case 7: return launch_ws<K, DP, 7, F16>(p, st);
-    case 8: return launch_ws<K, DP, 8, F16>(p, st);
+    case 1: return launch_ws<K, DP, 1, F16, RS>(p, st);
+    case 2: return launch_ws<K, DP, 2, F16, RS>(p, st);
+    case 3: return launch_ws<K, DP, 3, F16, RS>(p, st);
+    case 4: return launch_ws<K, DP, 4, F16, RS>(p, st);
+    case 5: return launch_ws<K, DP, 5, F16, RS>(p, st);
+    case 6: return launch_ws<K, DP, 6, F16, RS>(p, st);
+    case 7: return launch_ws<K, DP, 7, F16, RS>(p, st);
+    case 8: return launch_ws<K, DP, 8, F16, RS>(p, st);
   }
   return cudaErrorNotSupported;
+}
+
+template <int K, int DP, bool F16>
+cudaError_t by_b(int B, const DecArgs& p, cudaStream_t st) {
+  return p.rho != nullptr ? by_b_rs<K, DP, F16, true>(B, p, st)
+                          : by_b_rs<K, DP, F16, false>(B, p, st);
 }
 
 }  // namespace
@@ -610,10 +649,11 @@ bool decode_supported(fq_dtype yt, const Shape& s, const void* codes, const void
 
 cudaError_t launch_decode(const uint8_t* codes, const uint16_t* norms, int64_t n,
                           const Shape& s, const float* rot, const float* cb, void* y,
-                          fq_dtype yt, cudaStream_t st) {
+                          fq_dtype yt, cudaStream_t st, const uint16_t* rho, int rule) {
   if (n > (int64_t)INT32_MAX)  // tensor-map row coordinates are 32-bit
-    return launch_decode_generic(codes, norms, n, s, rot, cb, y, yt, st);
-  DecArgs p{n, rot, cb, codes, norms, y};
+    return launch_decode_generic(codes, norms, n, s, rot, cb, y, yt, st, Gather{nullptr, 0},
+                                 Rescale{rho, rule});
+  DecArgs p{n, rot, cb, codes, norms, y, rho, rule};
   const bool f16 = yt == FQ_F16;
   switch (s.k) {
     case 2: return f16 ? by_b<2, 64, true>(s.B, p, st) : by_b<2, 64, false>(s.B, p, st);

@@ -79,7 +79,25 @@ struct EncParams {
   const uint8_t* index;
   uint8_t* codes;
   uint16_t* norms;
+  uint16_t* rho;  // the rescale variant: rho = <z, zhat> per vector (fp16), else nullptr
 };
+
+// z_b . c of the codeword c whose table entry this lane reads (the table holds c for k = 2 and
+// -2c for k = 3, 4)
+template <int K>
+__device__ __forceinline__ float zdot_tbl(const void* __restrict__ tbl, int c,
+                                          const float (&zb)[K]) {
+  if constexpr (K == 2) {
+    const float2 t = reinterpret_cast<const float2*>(tbl)[c * 16];
+    return fmaf(zb[1], t.y, zb[0] * t.x);
+  } else if constexpr (K == 3) {
+    const float4 t = reinterpret_cast<const float4*>(tbl)[c * 8];
+    return -0.5f * fmaf(zb[2], t.z, fmaf(zb[1], t.y, zb[0] * t.x));
+  } else {
+    const float4 t = reinterpret_cast<const float4*>(tbl)[2 * c];
+    return -0.5f * fmaf(zb[3], t.w, fmaf(zb[2], t.z, fmaf(zb[1], t.y, zb[0] * t.x)));
+  }
+}
 
 // acc + lo^2 + hi^2 for the two fp16 values packed in hw (the products are exact)
 __device__ __forceinline__ float sq2_acc(uint32_t hw, float acc) {
@@ -278,7 +296,7 @@ __device__ __forceinline__ bool pipe_sync_or(int pipe, bool pred) {
   return r != 0;
 }
 
-template <int K, int DP, int B, bool GRID>
+template <int K, int DP, int B, bool GRID, bool RHO>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_kernel(const __grid_constant__ CUtensorMap xmap, EncParams p) {
   using C = EncCfg<K, DP, B>;
@@ -480,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fail = !ptx::mbar_wait(&mma_done[pipe], (uint32_t)i & 1u);
       ptx::tc_fence_after();
       const uint32_t bit0 = (uint32_t)lt * (C::P * 8);
+      float rho = 0.f;  // RHO: <z, zhat>, block by block
       const float2 r2 = make_float2(rinv, rinv);
       const float2 l2 = make_float2(kLoScale * rinv, kLoScale * rinv);
       // groups of G blocks: z = (D_hi + 2^-12 D_lo) / nu from tensor memory, nearest codewords
@@ -504,7 +523,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           float zb[K];
 #pragma unroll
           for (int a = 0; a < K; ++a) zb[a] = z[b * K + a];
-          v |= (uint64_t)search.find(zb) << (b * B);
+          const int c = search.find(zb);
+          v |= (uint64_t)c << (b * B);
+          if constexpr (RHO) rho += zdot_tbl<K>(tbl, c, zb);
         }
         if (nu > 0.f) or_bits(st, bit0 + (uint32_t)(gi * C::G * B), v);
       }
@@ -525,12 +546,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           float zb[K];
 #pragma unroll
           for (int a = 0; a < K; ++a) zb[a] = z[b * K + a];
-          v |= (uint64_t)search.find(zb) << (b * B);
+          const int c = search.find(zb);
+          v |= (uint64_t)c << (b * B);
+          if constexpr (RHO) rho += zdot_tbl<K>(tbl, c, zb);
         }
         if (nu > 0.f) or_bits(st, bit0 + (uint32_t)(C::NG * C::G * B), v);
       }
       const int64_t row = tile * kRows + lt;
-      if (row < p.n) p.norms[row] = f32_to_f16_bits(nu);
+      if (row < p.n) {
+        p.norms[row] = f32_to_f16_bits(nu);
+        if constexpr (RHO) p.rho[row] = f32_to_f16_bits(nu > 0.f ? rho : 1.f);  // zero: rho = 1
+      }
       ptx::tc_fence_before();
       // tensor memory is free for the next tile's MMA; the tile's records are complete
       if (pipe_sync_or(pipe, fail)) {
@@ -601,7 +627,7 @@ PFN_cuTensorMapEncodeTiled_v12000 enc_tensor_map_fn() {
   return fn;
 }
 
-template <int K, int DP, int B, bool GRID>
+template <int K, int DP, int B, bool GRID, bool RHO>
 cudaError_t launch_kernel(const void* x, const EncParams& p, cudaStream_t st) {
   using C = EncCfg<K, DP, B>;
   CUtensorMap map;
@@ -615,7 +641,7 @@ cudaError_t launch_kernel(const void* x, const EncParams& p, cudaStream_t st) {
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = encode_kernel<K, DP, B, GRID>;
+  auto kern = encode_kernel<K, DP, B, GRID, RHO>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -632,8 +658,12 @@ template <int K, int DP, int B>
 cudaError_t launch_rate(const void* x, const EncParams& p, cudaStream_t st) {
   // with an index, codebooks of 16 codewords and more search their grid candidate lists (3
   // candidates at N = 16 against 16 from registers); smaller ones keep the register brute force
-  if (p.index != nullptr && B >= 4) return launch_kernel<K, DP, B, true>(x, p, st);
-  return launch_kernel<K, DP, B, false>(x, p, st);
+  const bool grid = p.index != nullptr && B >= 4;
+  if (p.rho != nullptr)
+    return grid ? launch_kernel<K, DP, B, true, true>(x, p, st)
+                : launch_kernel<K, DP, B, false, true>(x, p, st);
+  return grid ? launch_kernel<K, DP, B, true, false>(x, p, st)
+              : launch_kernel<K, DP, B, false, false>(x, p, st);
 }
 
 template <int K, int DP>
@@ -667,10 +697,11 @@ bool encode_supported(fq_dtype xt, const Shape& s, const void* x, const void* co
 
 cudaError_t launch_encode(const void* x, fq_dtype, int64_t n, const Shape& s, const float* rot,
                           const float* cb, uint8_t* codes, uint16_t* norms, const void* index,
-                          cudaStream_t st) {
+                          cudaStream_t st, uint16_t* rho) {
   if (n > (int64_t)INT32_MAX)  // tensor-map row coordinates are 32-bit
-    return launch_encode_generic(x, FQ_F16, n, s, rot, cb, codes, norms, index, st);
-  EncParams p{n, s.N, rot, cb, static_cast<const uint8_t*>(index), codes, norms};
+    return launch_encode_generic(x, FQ_F16, n, s, rot, cb, codes, norms, index, st,
+                                 AppendMap{nullptr, 1, 0}, rho);
+  EncParams p{n, s.N, rot, cb, static_cast<const uint8_t*>(index), codes, norms, rho};
   switch (s.k) {
     case 2: return by_b<2, 64>(s.B, x, p, st);
     case 3: return by_b<3, 66>(s.B, x, p, st);

@@ -293,9 +293,12 @@ fq_status fq_encode_rho(const void* x, fq_dtype x_type, int64_t n, int d, int k,
   if (!aligned(x, x_type == FQ_F16 ? 2 : 4) || !aligned(norms, 2) || !aligned(rho, 2) ||
       !aligned(rot, 4) || !aligned(codebook, 4) || (search_index && !aligned(search_index, 8)))
     return FQ_ERR_ALIGNMENT;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (sm100::encode_supported(x_type, s, x, codes, norms))
+    return from_cuda(sm100::launch_encode(x, x_type, n, s, rot, codebook, codes, norms,
+                                          search_index, cs, rho));
   return from_cuda(launch_encode_generic(x, x_type, n, s, rot, codebook, codes, norms,
-                                         search_index, static_cast<cudaStream_t>(stream),
-                                         AppendMap{nullptr, 1, 0}, rho));
+                                         search_index, cs, AppendMap{nullptr, 1, 0}, rho));
 }
 
 fq_status fq_decode_rescaled(const uint8_t* codes, const uint16_t* norms, const uint16_t* rho,
@@ -313,9 +316,12 @@ fq_status fq_decode_rescaled(const uint8_t* codes, const uint16_t* norms, const 
   if (!aligned(norms, 2) || !aligned(rho, 2) || !aligned(rot, 4) || !aligned(codebook, 4) ||
       !aligned(y, y_type == FQ_F16 ? 2 : 4))
     return FQ_ERR_ALIGNMENT;
-  return from_cuda(launch_decode_generic(codes, norms, n, s, rot, codebook, y, y_type,
-                                         static_cast<cudaStream_t>(stream), Gather{nullptr, 0},
-                                         Rescale{rho, rule}));
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (sm100::decode_supported(y_type, s, codes, norms, y))
+    return from_cuda(sm100::launch_decode(codes, norms, n, s, rot, codebook, y, y_type, cs, rho,
+                                          rule));
+  return from_cuda(launch_decode_generic(codes, norms, n, s, rot, codebook, y, y_type, cs,
+                                         Gather{nullptr, 0}, Rescale{rho, rule}));
 }
 
 static fq_status prod_shape(int d, int N1, int* B1, int* P1) {

@@ -27,13 +27,18 @@ def _rows(n):
     return x
 
 
-@pytest.mark.parametrize("dp,k,N", [(66, 3, 64), (64, 2, 16), (64, 4, 8)])
-def test_rescale_rho_and_rules_match_the_oracle(dp, k, N):
+@pytest.mark.parametrize("dp,k,N,grid", [(66, 3, 64, None), (64, 2, 16, None), (64, 4, 8, None),
+                                         (66, 3, 64, (20, 8)), (64, 2, 256, (128, 4))])
+def test_rescale_rho_and_rules_match_the_oracle(dp, k, N, grid):
+    """rho and the decoder's S rules; fp16 rows of d = 64 take the tensor-core encode (with an
+    exact grid index: the grid search), others the generic kernels."""
     d = 64
     rot, cb = tables.rotation(dp, wl.ROT_SEED_V), tables.codebook(dp, k, N)
     x = _rows(1500)
     rt, ct = _dev(rot), _dev(cb)
-    codes, norms, rho = fq.fq_encode_rho(_dev(x), rt, ct, k, N)
+    ix = None if grid is None else \
+        _dev(fq.fq_build_search_index(cb, d, k, N, fq.FQ_INDEX_EXACT, grid[0], grid[1]))
+    codes, norms, rho = fq.fq_encode_rho(_dev(x), rt, ct, k, N, search_index=ix)
     torch.cuda.synchronize()
     enc, _ = fo.encode_rescaled(x, rot, cb, k)
     gidx = par.check_records_and_indices(par.to_np(codes), enc, N, dp // k)
