@@ -525,12 +525,23 @@ def attn_bench(torch, fq, timer, device, rank, hbm):
     cmean, cmin = cosine()
     gbs = attn_bytes / (us * 1e-6) / 1e9
     # random access: per-sequence lengths (random in [1, T]) and the step that appends its token
+    # (CUDA-graph replay like the full step: device time, no host launch overhead)
     w = wl.ATTN
     per_tok = attn_bytes / (w.batch * w.hkv * w.tokens)
-    us_len = _time_ms(torch, extra["launch_lengths"]) * 1e3
-    len_bytes = float(extra["lengths"].sum().item()) * w.hkv * per_tok
     extra["reset_append"](w.tokens // 2)
-    us_app = _time_ms(torch, extra["launch_append"], reps=50) * 1e3
+    extra["launch_lengths"]()   # eager once before capture (library set-up of each entry point)
+    extra["launch_append"]()
+    torch.cuda.synchronize()
+    g_len = timer.capture([extra["launch_lengths"]])
+    g_len.replay()
+    reps_len = timer.adaptive_reps([g_len], target_s=0.1, lo=20, hi=1000)
+    us_len = timer.time([g_len], reps_len) * 1e3 / reps_len
+    len_bytes = float(extra["lengths"].sum().item()) * w.hkv * per_tok
+    g_app = timer.capture([extra["launch_append"]])  # capture records the step, runs nothing
+    extra["reset_append"](w.tokens // 2)
+    torch.cuda.synchronize()
+    us_app = timer.time([g_app], 50) * 1e3 / 50
+    del g_len, g_app
     app_tokens = w.tokens // 2 + 26   # lengths advance by one per call: mean over the calls
     app_bytes = w.batch * w.hkv * app_tokens * per_tok
     return {"workload": wl.ATTN.name, "us_per_step": round(us, 2), "bytes_per_step": attn_bytes,

@@ -187,7 +187,7 @@ __device__ __forceinline__ void value_chunk(const uint4 (&e)[MV], bool hi, uint3
   o[3] = value_word<KV, MV, 4 * C8 + 3>(e, hi);
 }
 
-template <int G, int KB, int KV, int VB>
+template <int G, int KB, int KV, int VB, bool RAGGED>
 __global__ void __launch_bounds__(kThr, Cfg<G, KB, KV, VB>::MIN_CTAS)
     attn_partial_sm100(AttnArgs a) {
   using C = Cfg<G, KB, KV, VB>;
@@ -219,6 +219,18 @@ __global__ void __launch_bounds__(kThr, Cfg<G, KB, KV, VB>::MIN_CTAS)
   const int64_t t_end = (t_begin + a.tokens_per_split < len_b) ? t_begin + a.tokens_per_split : len_b;
   const int n_tiles = t_end > t_begin ? (int)((t_end - t_begin + kT - 1) / kT) : 0;
   const size_t kv_base = ((size_t)b * a.Hkv + g) * (size_t)a.T;
+  if constexpr (RAGGED) if (n_tiles == 0) {
+    // a split past its sequence's end: its empty partials (m = -inf, l = 0, acc = 0) and
+    // nothing else (no tensor memory, tables or queries); only with per-sequence lengths, so
+    // that the full step's kernel is not touched by the extra path
+    constexpr int dpv2 = C::DPV + 2;
+    for (int e = threadIdx.x; e < G * dpv2; e += kThr) {
+      const int h = e / dpv2, c = e % dpv2;
+      a.partials[(((size_t)b * a.Hq + (size_t)g * G + h) * a.splits + split) * dpv2 + c] =
+          c == 0 ? -INFINITY : 0.f;
+    }
+    return;
+  }
 
   // sources of tile i: key records, value records, key norms, value norms
   auto src_of = [&](int i) {
@@ -683,7 +695,12 @@ __global__ void __launch_bounds__(kThr, Cfg<G, KB, KV, VB>::MIN_CTAS)
 template <int G, int KB, int KV, int VB>
 cudaError_t launch(const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<G, KB, KV, VB>;
-  auto kern = attn_partial_sm100<G, KB, KV, VB>;
+  // the empty-split shortcut for per-sequence lengths is built for 8 query heads per kv head
+  // (the attention workloads' ratio); other ratios run the full kernel, which handles empty
+  // splits too
+  auto kern = attn_partial_sm100<G, KB, KV, VB, false>;
+  if constexpr (G == 8)
+    if (a.lengths != nullptr) kern = attn_partial_sm100<G, KB, KV, VB, true>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.splits, a.Hkv, a.B), kThr, C::SMEM, st>>>(a);
