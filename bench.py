@@ -812,6 +812,14 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+def e2e_chunks(n: int) -> int:
+    """Row chunks of the end-to-end step over n rows (K then V halves): as many as split both
+    halves evenly, up to 32 (the first upload and the last download are the only copies nothing
+    overlaps, about 1/chunks of the step each)."""
+    half = n // 2
+    return next(c for c in (32, 16, 8, 4, 2) if half % (c // 2) == 0)
+
+
 def e2e(torch, fq, run, args, device, world, dist, chunks=None):
     """Same metric through the public API with host buffers.  Every step copies the pinned host
     cache in, encodes, copies the records out, copies them back in, decodes and copies the fp16
@@ -822,9 +830,8 @@ def e2e(torch, fq, run, args, device, world, dist, chunks=None):
     shape, states = run.shape, run.step
     n, d = shape.n, shape.d
     half = n // 2
-    if chunks is None:  # as many as split K and V evenly, up to 32 (the first upload and the
-        # last download are the only copies nothing overlaps, about 1/chunks of the step each)
-        chunks = next(c for c in (32, 16, 8, 4, 2) if half % (c // 2) == 0)
+    if chunks is None:
+        chunks = e2e_chunks(n)
     per = half // (chunks // 2)
     assert per * chunks == n, "chunks must split the K and V halves evenly"
     xh = torch.from_numpy(run.host).pin_memory()

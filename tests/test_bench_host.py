@@ -70,3 +70,16 @@ def test_step_and_extra_rates_and_cpu_sample():
 def test_whole_job_rate_and_single_process_max():
     assert bench.whole_job_rate(4, 2.5e9, 10, 1000.0) == 4 * 2.5e9 * 10 / 1.0 / 1e9
     assert bench.max_over_ranks(None, None, 12.5, None) == 12.5
+
+
+def test_e2e_chunks_split_both_halves_evenly():
+    """The end-to-end step's row chunks split K and V evenly for every workload (and shrunken
+    sequence lengths), up to 32 chunks."""
+    from random_access_kv_fq_b200 import workloads as wl
+    sizes = [w.cache.n for w in wl.CODEC_WORKLOADS.values()] + [524288, 4096, 6, 2]
+    for n in sizes:
+        c = bench.e2e_chunks(n)
+        half = n // 2
+        assert c in (32, 16, 8, 4, 2) and half % (c // 2) == 0
+        assert (half // (c // 2)) * c == n
+    assert bench.e2e_chunks(wl.LARGE.cache.n) == 32
