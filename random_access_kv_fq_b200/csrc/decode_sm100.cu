@@ -22,6 +22,9 @@
 //               staging tile that one TMA tensor store per warp copies out; they first build
 //               the rotation operand, which the MMA warp waits for
 // so the copies, the gather of tile i + 1, the MMAs and the epilogue of tile i overlap.
+// The rescale variant (Block Sphere VQ key design 3, a template flag) scales each row by S nu
+// instead: its epilogue thread unpacks the row's record, sums |c|^2 of its codewords for the MSE
+// rule and reads the stored rho.
 // Every wait is bounded; a timed-out wait raises an abort flag that ends all roles.
 #include <cstdint>
 

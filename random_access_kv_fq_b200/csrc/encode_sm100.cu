@@ -18,6 +18,8 @@
 //            the shared-memory codebook), so the hot code stays small
 //   pack     each group's indices are OR-ed into the vector's record in shared memory; the
 //            tile's records leave with coalesced 16-byte stores.
+// The rescale variant (Block Sphere VQ key design 3, a template flag) also sums, block by block,
+// z_b . c of the chosen codeword from the same table and writes rho = <z, zhat> beside the norm.
 #include <cstdint>
 
 #include <cuda.h>
